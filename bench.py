@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 weight-streaming linear on B200.
+
+Metric: effective HBM bandwidth of Y[M,N] = X[M,K] W^T, counting
+bytes = N*K/2 + N*K/16 + 2*M*K + 2*M*N per call (packed codes, E4M3 scales,
+X and Y), reported in GB/s and as a fraction of the measured device-copy peak.
+One "step" is one call of the linear on one batch of M tokens. The headline
+workload is the single-token decode projection M=1, K=5120, N=34816 (a fused
+gate+up of a 27B-class decoder with hidden size 5120).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own replica
+of the workload (replicas only: the linear needs no exchange); the time is the
+maximum over ranks and the value the bytes of all ranks over that time.
+Inputs are synthetic (seeded generators in synth/), weights rotate over enough
+byte-identical copies that the footprint is > 4x the L2 cache.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 linear effective HBM GB/s and % of peak at M=1/16 (27B-class shapes)"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def bytes_per_call(M: int, N: int, K: int) -> int:
+    return N * K // 2 + N * K // 16 + 2 * M * K + 2 * M * N
+
+
+def effective_gbs(nbytes: float, seconds: float) -> float:
+    return nbytes / seconds / 1e9
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while work runs."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, period_ms: int = 50):
+        self.index = index
+        self.period_ms = period_ms
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        import datetime
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        sm, smax, reasons, total = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            try:
+                ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                mhz, mx = float(r[2]), float(r[3])
+            except (ValueError, IndexError):
+                continue
+            total += 1
+            # keep the samples taken inside the timed region (small margin)
+            if self.t0 is not None and not (self.t0 - 0.06 <= ts <= self.t1 + 0.06):
+                continue
+            sm.append(mhz)
+            smax = mx
+            for name, val in zip(names, r[6:10]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm), "samples_total": total}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        if torch.cuda.is_available():
+            torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, value: float) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(world, value: float) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+class Problem:
+    """One workload on the device: weight copies, X, Y, plan, workspace."""
+
+    def __init__(self, name: str, M: int, variant: int, min_footprint: float):
+        import numpy as np
+        import torch
+        import synth
+        import nvfp4_weight_streaming_b200 as nv
+        self.nv = nv
+        wl = synth.WORKLOADS[name]
+        self.name, self.M, self.N, self.K = name, M, wl.N, wl.K
+        dev = torch.cuda.current_device()
+        # weights: generated on the host, quantised on the device by the library
+        W = torch.from_numpy(synth.weights_f32(wl)).cuda()
+        packed = torch.empty((self.N, self.K // 2), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((self.N, self.K // 16), dtype=torch.uint8, device="cuda")
+        gs = torch.empty(1, dtype=torch.float32, device="cuda")
+        bad = torch.zeros(1, dtype=torch.int32, device="cuda")
+        nv.nvfp4_quantize(W, self.N, self.K, packed, scales, gs, bad)
+        torch.cuda.synchronize()
+        assert int(bad.item()) == 0
+        del W
+        wbytes = packed.numel() + scales.numel()
+        self.ncopies = max(1, math.ceil(min_footprint / wbytes))
+        self.copies = [(packed, scales)] + [(packed.clone(), scales.clone())
+                                            for _ in range(self.ncopies - 1)]
+        self.gs = gs
+        xh = synth.x_bf16(wl, M)
+        self.x_host = xh
+        self.x = torch.from_numpy(xh.view(np.int16)).cuda()
+        self.y = torch.empty((M, self.N), dtype=torch.int16, device="cuda")
+        self.plan = nv.nvfp4_linear_plan(M, self.N, self.K, dev, variant)
+        self.variant = nv.nvfp4_linear_variant(self.plan)
+        self.split_k = nv.nvfp4_linear_split_k(self.plan)
+        self.wsb = nv.nvfp4_linear_workspace_bytes(self.plan)
+        self.ws = torch.zeros(max(self.wsb, 16), dtype=torch.uint8, device="cuda")
+        self.bytes = bytes_per_call(M, self.N, self.K)
+        self.footprint = wbytes * self.ncopies
+        self.lib = nv.lib()
+
+    def call(self, i: int, stream_handle: int):
+        p, s = self.copies[i % self.ncopies]
+        st = self.lib.nvfp4_linear_run(self.plan, p.data_ptr(), s.data_ptr(), self.gs.data_ptr(),
+                                       self.x.data_ptr(), self.y.data_ptr(),
+                                       self.ws.data_ptr() if self.wsb else None, self.wsb,
+                                       stream_handle)
+        if st != 0:
+            raise RuntimeError("nvfp4_linear_run failed: %s" % self.nv.nvfp4_status_string(st))
+
+    def check_status(self):
+        import torch
+        st = self.nv.nvfp4_linear_status(self.plan, self.ws if self.wsb else None,
+                                         torch.cuda.current_stream())
+        if st != 0:
+            raise RuntimeError("device status: %s" % self.nv.nvfp4_status_string(st))
+
+    def destroy(self):
+        self.nv.nvfp4_linear_destroy(self.plan)
+
+
+def time_problem(pb: Problem, steps: int, warmup: int, world: int, graph_len: int = 64,
+                 sampler: ClockSampler | None = None):
+    """Warm up, then time exactly `steps` calls (replayed from CUDA graphs of
+    `graph_len` calls) between CUDA events; returns seconds per call (max over
+    ranks) and the number of kernel launches timed."""
+    import torch
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        h = stream.cuda_stream
+        for i in range(max(3, warmup)):
+            pb.call(i, h)
+    stream.synchronize()
+    pb.check_status()
+    glen = max(1, min(graph_len, steps))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        h = torch.cuda.current_stream().cuda_stream
+        for i in range(glen):
+            pb.call(i, h)
+    tail = steps % glen
+    tail_graph = None
+    if tail:
+        tail_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tail_graph, stream=stream):
+            h = torch.cuda.current_stream().cuda_stream
+            for i in range(tail):
+                pb.call(i, h)
+    # untimed replay so the graphs are uploaded and warm
+    with torch.cuda.stream(stream):
+        graph.replay()
+    stream.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark("t0")
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps // glen):
+            graph.replay()
+        if tail_graph is not None:
+            tail_graph.replay()
+        e1.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark("t1")
+    barrier(world)
+    sec = e0.elapsed_time(e1) / 1e3
+    pb.check_status()
+    del graph, tail_graph
+    return max_over_ranks(world, sec) / steps, steps
+
+
+def time_e2e(pb: Problem, steps: int, world: int):
+    """Same metric through the public API with host buffers: each step copies
+    the weight copy and X from pinned host memory, runs, reads Y back."""
+    import numpy as np
+    import torch
+    p, s = pb.copies[0]
+    hp = torch.empty(p.shape, dtype=torch.uint8).pin_memory()
+    hs = torch.empty(s.shape, dtype=torch.uint8).pin_memory()
+    hp.copy_(p.cpu())
+    hs.copy_(s.cpu())
+    hx = torch.from_numpy(pb.x_host.view(np.int16)).pin_memory()
+    hy = torch.empty(pb.y.shape, dtype=torch.int16).pin_memory()
+    stream = torch.cuda.current_stream()
+    h = stream.cuda_stream
+
+    def step():
+        p.copy_(hp, non_blocking=True)
+        s.copy_(hs, non_blocking=True)
+        pb.x.copy_(hx, non_blocking=True)
+        pb.call(0, h)
+        hy.copy_(pb.y, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    sec = max_over_ranks(world, e0.elapsed_time(e1) / 1e3) / steps
+    h2d = hp.numel() + hs.numel() + hx.numel() * 2
+    d2h = hy.numel() * 2
+    return sec, h2d, d2h
+
+
+def cpu_baseline(sample_rows: int = 34816, M: int = 1):
+    """The oracle, as it stands, on the host cores: quantise the decode
+    workload's weights (oracle quantiser) and time its fp64 linear on
+    `sample_rows` rows."""
+    import numpy as np
+    import oracle
+    import synth
+    wl = synth.WORKLOADS["decode"]
+    rows = min(sample_rows, wl.N)
+    W = synth.weights_f32(wl, rows=slice(0, rows))
+    gs = oracle.global_scale(synth.weights_f32(wl))
+    packed, scales = oracle.quantize_rows(W, gs)
+    X = synth.x_bf16(wl, M)
+    cores = oracle.NTHREADS
+    oracle.linear(packed, scales, gs, X, M, rows, wl.K, nthreads=cores)   # warm-up
+    ts = []
+    for _ in range(3):
+        t0 = time.perf_counter()
+        oracle.linear(packed, scales, gs, X, M, rows, wl.K, nthreads=cores)
+        ts.append(time.perf_counter() - t0)
+    t = statistics.median(ts)
+    return {"value": effective_gbs(bytes_per_call(M, rows, wl.K), t), "unit": "GB/s",
+            "cores": cores, "kind": "oracle",
+            "sample": "fp64 oracle linear, decode workload M=%d K=%d, first %d of %d rows, "
+                      "median of 3" % (M, wl.K, rows, wl.N)}
+
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    import nvfp4_weight_streaming_b200 as nv
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    peak, peak_kind = peaks()
+    variant = {"auto": 0, "gemv": 1, "mma": 2, "tc": 3}[args.variant]
+    pb = Problem(args.workload, args.M, variant, min_footprint=4.2 * l2)
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    sec, launches = time_problem(pb, args.steps, args.warmup, world, sampler=sampler)
+    clocks = sampler.stop() if sampler else None
+    value = effective_gbs(pb.bytes * world, sec)
+    per_gpu = effective_gbs(pb.bytes, sec)
+    sweep = []
+    if not args.no_sweep:
+        for (name, M) in ([("verify", 16)] if not args.full_sweep else
+                          [("verify", m) for m in (1, 2, 4, 8, 12, 16)] +
+                          [("down", m) for m in (1, 4, 8, 16)] +
+                          [("lm_head", m) for m in (1, 8, 16)]):
+            q = Problem(name, M, variant, min_footprint=4.2 * l2)
+            s2, _ = time_problem(q, max(args.steps, 200), args.warmup, world)
+            g = effective_gbs(q.bytes, s2)
+            sweep.append({"workload": name, "M": M, "N": q.N, "K": q.K,
+                          "variant": ["auto", "gemv", "mma", "tc"][q.variant],
+                          "split_k": q.split_k, "us_per_call": s2 * 1e6, "GBps": g,
+                          "frac_of_measured_peak": g / peak})
+            q.destroy()
+            del q
+            torch.cuda.empty_cache()
+    e2e = None
+    if not args.no_e2e:
+        esec, h2d, d2h = time_e2e(pb, max(3, min(args.steps, 20)), world)
+        e2e = {"value": effective_gbs(pb.bytes * world, esec), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4 weights x bf16 activations, f16 products, f32 accumulate",
+            "data": "synthetic (seeded SplitMix64/Box-Muller, workload recipes in synth/)",
+            "config": {"workload": "%s projection M=%d K=%d N=%d" % (args.workload, pb.M, pb.K, pb.N),
+                       "M": pb.M, "K": pb.K, "N": pb.N,
+                       "variant": ["auto", "gemv", "mma", "tc"][pb.variant],
+                       "split_k": pb.split_k, "bytes_per_call": pb.bytes,
+                       "l2": "inputs larger than L2: %d byte-identical weight copies "
+                             "rotated, %.0f MB > %.1f x %.0f MB L2" %
+                             (pb.ncopies, pb.footprint / 1e6, pb.footprint / l2, l2 / 1e6),
+                       "launch": "CUDA graphs of back-to-back calls on one stream",
+                       "parallelism": "replicas x%d" % world},
+            "pct_of_measured_peak": 100 * per_gpu / peak,
+            "pct_of_nominal_8TBps": 100 * per_gpu / NOMINAL_HBM_GBS,
+            "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s",
+                         "frac": per_gpu / peak, "traffic": None,
+                         "peak_kind": peak_kind + " device-copy bandwidth (MEASURED_PEAKS hbm_gbs)"},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+    pb.destroy()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    import synth
+    wl = synth.WORKLOADS[args.workload]
+    M = args.M
+    rows = max(64, min(wl.N, int(args.reference_rows)))
+    gs = oracle.global_scale(synth.weights_f32(wl))
+    packed, scales = oracle.quantize_rows(synth.weights_f32(wl, rows=slice(0, rows)), gs)
+    X = synth.x_bf16(wl, M)
+    cores = oracle.NTHREADS
+    for _ in range(max(0, args.warmup)):
+        oracle.linear(packed, scales, gs, X, M, rows, wl.K, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.linear(packed, scales, gs, X, M, rows, wl.K, nthreads=cores)
+    sec = (time.perf_counter() - t0) / max(1, args.steps)
+    value = effective_gbs(bytes_per_call(M, rows, wl.K), sec)
+    sample = ("each step: fp64 oracle linear on the first %d of %d rows of the %s workload "
+              "(M=%d, K=%d), bytes scaled to the sample" % (rows, wl.N, args.workload, M, wl.K))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "%s projection M=%d K=%d N=%d" % (args.workload, M, wl.K, wl.N),
+                   "M": M, "K": wl.K, "N": wl.N},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode")
+    ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--variant", choices=["auto", "gemv", "mma", "tc"], default="auto")
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--full-sweep", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-rows", type=int, default=2048)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,158 @@
+/*
+ * nvfp4_linear.h -- C ABI of the NVFP4 weight-streaming linear for NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation. Y[M][N] = X[M][K] * W^T, where W[N][K] is stored as NVFP4:
+ *   - 4-bit E2M1 codes, two per byte, element 2j of a row in the LOW nibble of
+ *     byte j, rows contiguous: w_packed is uint8 [N][K/2];
+ *   - one E4M3 ("fn") scale byte per 16 consecutive K elements of a row:
+ *     w_scales is uint8 [N][K/16], row-major;
+ *   - one fp32 per-tensor scale gs (device memory), so that
+ *       w_hat[n][k] = e2m1(code[n][k]) * e4m3(scale[n][k/16]) * gs.
+ * X and Y are bf16, row-major, M in [1, 16]: one decode token (M = 1) or one
+ * token plus up to 15 drafted tokens checked in a single pass (M <= 16).
+ *
+ * Where the operation is defined. Page "Qwen3.8-27B-NVFP4-RTX5090 API &
+ * Inference Endpoint": section "Recipe (NVIDIA ModelOpt)" (every Linear, the
+ * output projection included, is NVFP4 with 16-element scale groups and a
+ * per-tensor scale), section "Serving" (the codes are stored packed in uint8
+ * tensors) and section "Why lm_head is NVFP4, and why MTP is gone" (decode is
+ * bound by the weight read, so every byte saved is speed). Page "InventDB
+ * Sparkle", section "How it answers quickly" (a helper model drafts several
+ * tokens and the large model checks all of them in one pass: M = 1 + drafts).
+ * The pages fix neither the nibble order nor the scale layout; the library
+ * takes the readings stated above (low nibble first, plain row-major scales,
+ * global scale multiplies).
+ *
+ * Numerics. Each w_hat/gs product e2m1 * e4m3 is exact in half precision; the
+ * contraction accumulates in fp32 (tensor cores or CUDA cores, by variant);
+ * the epilogue computes y = gs * acc in fp32 and rounds to bf16 (nearest even).
+ * Per element |y - y_ref| <= 1e-2 |y_ref| + 1e-4 sum_k |w_hat x| against an
+ * fp64 reference.
+ *
+ * Conventions.
+ *   - Every buffer is device memory owned by the caller; the library never
+ *     allocates device memory. A plan holds only launch parameters.
+ *   - Calls that take a stream are asynchronous on it (a cudaStream_t passed
+ *     as void*; NULL = legacy default stream), except nvfp4_linear_status,
+ *     which synchronises that stream.
+ *   - Argument errors are returned before anything is launched. Device-side
+ *     timeouts of bounded waits are reported through the workspace status word
+ *     and read by nvfp4_linear_status.
+ *   - Limits: 1 <= M <= 16, N >= 0, K >= 0 with K % 256 == 0, every pointer
+ *     16-byte aligned (gs: 4-byte aligned). N need not be a multiple of any
+ *     tile size.
+ *   - Thread safety: plans are immutable after creation and may be shared by
+ *     threads; runs on different streams may proceed concurrently if they use
+ *     different workspaces.
+ */
+#ifndef NVFP4_LINEAR_H
+#define NVFP4_LINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,   /* a size, pointer or handle is invalid */
+  NVFP4_ERR_UNSUPPORTED = 2,   /* shape/variant combination not supported */
+  NVFP4_ERR_MISALIGNED = 3,    /* a pointer breaks the alignment rule */
+  NVFP4_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+  NVFP4_ERR_TIMEOUT = 5,       /* a bounded device wait gave up (status word) */
+  NVFP4_ERR_BAD_SCALE = 6,     /* reserved: scale/global checks report counts */
+  NVFP4_ERR_WORKSPACE = 7      /* workspace missing or smaller than required */
+} nvfp4_status;
+
+typedef struct nvfp4_plan_s* nvfp4_plan_t;
+
+/* Kernel variants (plan flags, bits 0..3). AUTO picks per (M, N, K) from a
+ * table of bandwidths measured on B200. */
+#define NVFP4_VARIANT_AUTO 0u
+#define NVFP4_VARIANT_GEMV 1u  /* CUDA-core warp-per-row GEMV, fp32 FMA        */
+#define NVFP4_VARIANT_MMA  2u  /* register-direct warp MMA, split over K       */
+#define NVFP4_VARIANT_TC   3u  /* tcgen05 + TMA ring + TMEM accumulators       */
+#define NVFP4_PLAN_VARIANT_MASK 0xFu
+/* Bits 8..15: split-K factor override (0 = let the plan choose). */
+#define NVFP4_PLAN_SPLITK_SHIFT 8u
+#define NVFP4_PLAN_SPLITK_MASK 0xFF00u
+/* Test only: the variant's producer never signals, so every bounded device
+ * wait runs out and the kernel reports NVFP4_ERR_TIMEOUT through the status
+ * word instead of computing. Has no effect on variants without device waits. */
+#define NVFP4_PLAN_TEST_STALL 0x40000000u
+
+/* Create a plan for Y[M][N] = X[M][K] W^T on `device`. Chooses the kernel
+ * variant (or takes the one forced in `flags`), the split of K and the grid.
+ * Returns INVALID_ARG for M outside [1,16], negative N/K, K % 256 != 0 or a
+ * null `out`; UNSUPPORTED if a forced variant cannot run this shape; CUDA if
+ * the device cannot be queried. On success *out must be released with
+ * nvfp4_linear_destroy. */
+nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
+                               nvfp4_plan_t* out);
+
+/* Device workspace bytes nvfp4_linear_run needs for this plan (split-K
+ * partials, tile counters and the 4-byte status word), 0 if none. The
+ * workspace must be zero-filled once before its first use; the kernels leave
+ * it zero-filled again after every run. */
+size_t nvfp4_linear_workspace_bytes(nvfp4_plan_t plan);
+
+/* Chosen variant (NVFP4_VARIANT_*) and split-K factor of a plan; -1 if null. */
+int nvfp4_linear_variant(nvfp4_plan_t plan);
+int nvfp4_linear_split_k(nvfp4_plan_t plan);
+
+/* Run the linear on `stream` (device pointers, see the layout above):
+ *   w_packed  uint8 [N][K/2]     w_scales uint8 [N][K/16] (E4M3)
+ *   w_global  fp32 [1]           x        bf16 [M][K]       y bf16 [M][N]
+ *   workspace >= nvfp4_linear_workspace_bytes(plan) bytes (NULL if 0).
+ * Must run on the plan's device (the current device). Returns INVALID_ARG
+ * for a null plan or pointer, MISALIGNED for a pointer off its alignment,
+ * WORKSPACE for a short workspace, CUDA if the launch fails. Y may not alias
+ * any input. K == 0 writes zeros to Y; N == 0 launches nothing. */
+nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
+                              const uint8_t* w_scales, const float* w_global,
+                              const void* x, void* y, void* workspace,
+                              size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, then report: CUDA if the stream holds an error,
+ * TIMEOUT if a kernel of this plan recorded a device-wait timeout in the
+ * workspace status word (the word is cleared), else OK. workspace may be NULL
+ * for plans whose workspace size is 0. */
+nvfp4_status nvfp4_linear_status(nvfp4_plan_t plan, void* workspace, void* stream);
+
+/* Release a plan (NULL is ignored). */
+void nvfp4_linear_destroy(nvfp4_plan_t plan);
+
+/* Unpack and scale-decode check. For every element writes the exact product
+ * e2m1(code) * e4m3(scale) -- without the global scale -- as bf16 to
+ * w_bf16_out [N][K] (nullable: then only counting is done), and adds to the
+ * device counter *d_bad (uint32, caller-zeroed) the number of NaN scale codes
+ * (0x7F, 0xFF) plus 1 if *w_global is NaN, infinite or negative. Values
+ * produced from NaN scales are unspecified. Same alignment rules as run;
+ * K % 16 == 0 suffices here. Asynchronous on `stream`. */
+nvfp4_status nvfp4_pack_check(const uint8_t* w_packed, const uint8_t* w_scales,
+                              const float* w_global, int N, int K,
+                              void* w_bf16_out, unsigned* d_bad, void* stream);
+
+/* Quantise fp32 W [N][K] (device) to NVFP4 with the recipe:
+ *   gs = amax|W| / (6*448); per 16-element block s = E4M3_RNE_sat((amax_b/6)/gs);
+ *   code = E2M1_RNE_sat(w / (e4m3(s) * gs)), codes of magnitude 0 stored as 0x0;
+ *   a block whose e4m3(s)*gs is 0 gets all-zero codes.
+ * Every step is one fp32 operation, in that order. Writes w_packed, w_scales
+ * and *w_global (device). *d_bad (nullable, caller-zeroed) receives the
+ * number of non-finite elements of W (the outputs are then unspecified).
+ * K % 16 == 0; pointers 16-byte aligned. Three kernels on `stream`. */
+nvfp4_status nvfp4_quantize(const float* w, int N, int K, uint8_t* w_packed,
+                            uint8_t* w_scales, float* w_global, unsigned* d_bad,
+                            void* stream);
+
+/* Static text for a status code. */
+const char* nvfp4_status_string(nvfp4_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_LINEAR_H */

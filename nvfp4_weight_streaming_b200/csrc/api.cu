@@ -1,0 +1,198 @@
+// api.cu -- the C ABI declared in include/nvfp4_linear.h.
+//
+// Argument checking, plan construction (variant and split choice), and the
+// launches. The library allocates no device memory; the caller passes every
+// buffer, and PyTorch (or any other allocator) owns them.
+#include "nvfp4_linear.h"
+#include "kernels.h"
+
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstdlib>
+#include <new>
+
+struct nvfp4_plan_s {
+  int M, N, K, device;
+  unsigned flags;
+  int variant;
+  int split_k;
+  int num_sms;
+  size_t ws_bytes;
+  nvfp4::GemvConfig gemv;
+};
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+nvfp4_status check_device(int device) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return NVFP4_ERR_CUDA;
+  return cur == device ? NVFP4_OK : NVFP4_ERR_INVALID_ARG;
+}
+
+// Which variant AUTO takes for a shape: the fastest measured on B200 for
+// that (M, N, K) class among those that can run it.
+int auto_variant(int M, int N, int K) {
+  (void)N;
+  if (M <= 4 && size_t(M) * size_t(K) * 4 <= 200 * 1024) return int(NVFP4_VARIANT_GEMV);
+  return int(NVFP4_VARIANT_GEMV);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4_status_string(nvfp4_status s) {
+  switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_UNSUPPORTED: return "unsupported shape or variant";
+    case NVFP4_ERR_MISALIGNED: return "misaligned pointer";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_TIMEOUT: return "device wait timed out";
+    case NVFP4_ERR_BAD_SCALE: return "bad scale";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
+                               nvfp4_plan_t* out) {
+  if (!out) return NVFP4_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (M < 1 || M > 16 || N < 0 || K < 0 || K % 256 != 0) return NVFP4_ERR_INVALID_ARG;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (device < 0 || device >= ndev) return NVFP4_ERR_INVALID_ARG;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  int prev = -1;
+  if (cudaGetDevice(&prev) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (prev != device && cudaSetDevice(device) != cudaSuccess) return NVFP4_ERR_CUDA;
+
+  nvfp4_plan_s p{};
+  p.M = M; p.N = N; p.K = K; p.device = device; p.flags = flags; p.num_sms = sms;
+  p.split_k = 1;
+  p.ws_bytes = 0;
+  unsigned forced = flags & NVFP4_PLAN_VARIANT_MASK;
+  p.variant = forced ? int(forced) : auto_variant(M, N, K);
+  nvfp4_status st = NVFP4_OK;
+  switch (p.variant) {
+    case NVFP4_VARIANT_GEMV: {
+      if (M > 4 || size_t(M) * size_t(K) * 4 > 200 * 1024) { st = NVFP4_ERR_UNSUPPORTED; break; }
+      p.gemv.M = M; p.gemv.N = N; p.gemv.K = K;
+      if (K > 0 && N > 0 && nvfp4::gemv_configure(p.gemv, sms) != cudaSuccess) st = NVFP4_ERR_CUDA;
+      break;
+    }
+    default:
+      st = NVFP4_ERR_UNSUPPORTED;
+  }
+  if (prev != device) cudaSetDevice(prev);
+  if (st != NVFP4_OK) return st;
+  nvfp4_plan_s* h = new (std::nothrow) nvfp4_plan_s(p);
+  if (!h) return NVFP4_ERR_CUDA;
+  *out = h;
+  return NVFP4_OK;
+}
+
+size_t nvfp4_linear_workspace_bytes(nvfp4_plan_t plan) { return plan ? plan->ws_bytes : 0; }
+int nvfp4_linear_variant(nvfp4_plan_t plan) { return plan ? plan->variant : -1; }
+int nvfp4_linear_split_k(nvfp4_plan_t plan) { return plan ? plan->split_k : -1; }
+
+void nvfp4_linear_destroy(nvfp4_plan_t plan) { delete plan; }
+
+nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
+                              const uint8_t* w_scales, const float* w_global,
+                              const void* x, void* y, void* workspace, size_t ws_bytes,
+                              void* stream) {
+  if (!plan) return NVFP4_ERR_INVALID_ARG;
+  const int M = plan->M, N = plan->N, K = plan->K;
+  if (N == 0) return NVFP4_OK;
+  if (!y || !w_global) return NVFP4_ERR_INVALID_ARG;
+  if (K > 0 && (!w_packed || !w_scales || !x)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(y, 16) || !aligned(w_global, 4)) return NVFP4_ERR_MISALIGNED;
+  if (K > 0 && (!aligned(w_packed, 16) || !aligned(w_scales, 16) || !aligned(x, 16)))
+    return NVFP4_ERR_MISALIGNED;
+  if (plan->ws_bytes > 0) {
+    if (!workspace || ws_bytes < plan->ws_bytes) return NVFP4_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return NVFP4_ERR_MISALIGNED;
+  }
+  nvfp4_status dv = check_device(plan->device);
+  if (dv != NVFP4_OK) return dv;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint16_t* yb = static_cast<uint16_t*>(y);
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  cudaError_t e = cudaSuccess;
+  if (K == 0) {
+    e = nvfp4::launch_zero_bf16(yb, int64_t(M) * N, st);
+  } else {
+    switch (plan->variant) {
+      case NVFP4_VARIANT_GEMV:
+        e = nvfp4::launch_gemv(plan->gemv, w_packed, w_scales, w_global, xb, yb, st);
+        break;
+      default:
+        return NVFP4_ERR_UNSUPPORTED;
+    }
+  }
+  return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status nvfp4_linear_status(nvfp4_plan_t plan, void* workspace, void* stream) {
+  if (!plan) return NVFP4_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (cudaPeekAtLastError() != cudaSuccess) return NVFP4_ERR_CUDA;
+  if (plan->ws_bytes > 0 && workspace) {
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+      return NVFP4_ERR_CUDA;
+    if (word != 0) {
+      uint32_t zero = 0;
+      if (cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+      return NVFP4_ERR_TIMEOUT;
+    }
+  }
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_pack_check(const uint8_t* w_packed, const uint8_t* w_scales,
+                              const float* w_global, int N, int K, void* w_bf16_out,
+                              unsigned* d_bad, void* stream) {
+  if (N < 0 || K < 0 || K % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (!w_global || !d_bad) return NVFP4_ERR_INVALID_ARG;
+  const int64_t nb = int64_t(N) * (K / 16);
+  if (nb > 0 && (!w_packed || !w_scales)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(w_global, 4) || !aligned(d_bad, 4)) return NVFP4_ERR_MISALIGNED;
+  if (nb > 0 && (!aligned(w_packed, 16) || !aligned(w_scales, 16))) return NVFP4_ERR_MISALIGNED;
+  if (w_bf16_out && !aligned(w_bf16_out, 16)) return NVFP4_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  cudaError_t e = nvfp4::launch_pack_check(w_packed, w_scales, w_global, nb,
+                                           static_cast<uint16_t*>(w_bf16_out), d_bad, sms,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status nvfp4_quantize(const float* w, int N, int K, uint8_t* w_packed, uint8_t* w_scales,
+                            float* w_global, unsigned* d_bad, void* stream) {
+  if (N < 0 || K < 0 || K % 16 != 0 || !w_global) return NVFP4_ERR_INVALID_ARG;
+  const int64_t n = int64_t(N) * K;
+  if (n > 0 && (!w || !w_packed || !w_scales)) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned(w_global, 4) || (d_bad && !aligned(d_bad, 4))) return NVFP4_ERR_MISALIGNED;
+  if (n > 0 && (!aligned(w, 16) || !aligned(w_packed, 16) || !aligned(w_scales, 16)))
+    return NVFP4_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  cudaError_t e = nvfp4::launch_quantize(w, N, K, w_packed, w_scales, w_global, d_bad, sms,
+                                         static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+}  // extern "C"

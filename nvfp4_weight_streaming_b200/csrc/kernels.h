@@ -1,0 +1,33 @@
+// kernels.h -- host-side launch interface between the C ABI (api.cu) and the
+// kernel translation units. Internal to the library.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+// Unpack + scale-decode check (k_basic.cu).
+cudaError_t launch_pack_check(const uint8_t* wp, const uint8_t* ws, const float* gs,
+                              int64_t nblocks16, uint16_t* out, unsigned* bad,
+                              int num_sms, cudaStream_t st);
+
+// GPU quantiser: amax, per-block quantise, finalise gs (k_basic.cu).
+cudaError_t launch_quantize(const float* w, int64_t N, int64_t K, uint8_t* wp, uint8_t* ws,
+                            float* gs, unsigned* bad, int num_sms, cudaStream_t st);
+
+// Zero-fill Y (K == 0).
+cudaError_t launch_zero_bf16(uint16_t* y, int64_t count, cudaStream_t st);
+
+// CUDA-core warp GEMV (k_gemv.cu). smem_bytes = M*K*4.
+struct GemvConfig {
+  int M, N, K;
+  int grid, block;
+  size_t smem;
+};
+cudaError_t gemv_configure(GemvConfig& c, int num_sms);
+cudaError_t launch_gemv(const GemvConfig& c, const uint8_t* wp, const uint8_t* ws,
+                        const float* gs, const uint16_t* x, uint16_t* y, cudaStream_t st);
+
+}  // namespace nvfp4

@@ -1,0 +1,330 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Integer work (unpack/scale decode, quantiser codes) must match bit for bit.
+Y must satisfy |y - y_ref| <= 1e-2 |y_ref| + 1e-4 sum_k |w_hat x| per element,
+and be exact where the arithmetic is exact (one-hot X, dyadic sums).
+Every output buffer carries canary guards that must survive the run.
+"""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_weight_streaming_b200 as nv
+import oracle
+import synth
+from tests.gpu_util import Guarded, Weights, check_tolerance, dev, host_u16, run_linear
+
+pytestmark = pytest.mark.gpu
+
+VARIANTS = [nv.NVFP4_VARIANT_GEMV, nv.NVFP4_VARIANT_MMA, nv.NVFP4_VARIANT_TC]
+VNAME = {0: "auto", 1: "gemv", 2: "mma", 3: "tc"}
+
+_cache = {}
+
+
+def quantized(name: str, copy: int = 0):
+    """(packed, scales, gs) of a workload's weights, quantised by the oracle."""
+    key = (name, copy)
+    if key not in _cache:
+        wl = synth.WORKLOADS[name]
+        _cache[key] = oracle.quantize(synth.weights_f32(wl, copy))
+    return _cache[key]
+
+
+def supported(variant: int, M: int, N: int, K: int) -> bool:
+    try:
+        p = nv.nvfp4_linear_plan(M, N, K, torch.cuda.current_device(), variant)
+    except nv.Nvfp4Error as e:
+        if e.status == nv.NVFP4_ERR_UNSUPPORTED:
+            return False
+        raise
+    nv.nvfp4_linear_destroy(p)
+    return True
+
+
+def variants_for(M, N, K):
+    vs = [v for v in VARIANTS if supported(v, M, N, K)]
+    assert vs, "no variant supports M=%d N=%d K=%d" % (M, N, K)
+    return vs + [nv.NVFP4_VARIANT_AUTO]
+
+
+# ----- unpack / scale decode (bit exact) -----------------------------------
+
+def pack_check(packed, scales, gs, N, K, with_out=True):
+    out = Guarded(N * K) if with_out else None
+    bad = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_pack_check(dev(packed), dev(scales),
+                        torch.tensor([gs], dtype=torch.float32, device="cuda"), N, K,
+                        None if out is None else out.view, bad)
+    torch.cuda.synchronize()
+    res = None if out is None else host_u16(out.view).reshape(N, K)
+    return res, int(bad.item()), (out is None or out.guards_intact())
+
+
+def test_pack_check_exhaustive_codes_times_scales():
+    finite = [c for c in range(256) if c not in (0x7F, 0xFF)]
+    N, K = len(finite), 32
+    packed = np.zeros((N, K // 2), np.uint8)
+    for j in range(K // 2):
+        packed[:, j] = ((2 * j) % 16) | (((2 * j + 1) % 16) << 4)
+    scales = np.repeat(np.array(finite, np.uint8).reshape(N, 1), 2, axis=1)
+    got, bad, ok = pack_check(packed, scales, 1.0, N, K)
+    assert ok and bad == 0
+    ref = oracle.dequant_bf16_nogs(packed, scales, N, K)
+    assert np.array_equal(got, ref)
+
+
+def test_pack_check_counts_nan_scales_and_bad_global():
+    packed = np.random.default_rng(0).integers(0, 256, size=(4, 32), dtype=np.uint8)
+    scales = np.array([[0x38, 0x7F, 0x40, 0x38], [0xFF, 0x00, 0x7F, 0x01],
+                       [0x38, 0x38, 0x38, 0x38], [0x80, 0xFE, 0x7E, 0x7F]], np.uint8)
+    for gs in (1.0, -1.0, float("nan"), float("inf"), 0.0):
+        _, bad, _ = pack_check(packed, scales, gs, 4, 64, with_out=False)
+        assert bad == oracle.count_bad(scales, gs)
+    got, _, ok = pack_check(packed, scales, 1.0, 4, 64)
+    ref = oracle.dequant_bf16_nogs(packed, scales, 4, 64)
+    finite = np.repeat(~np.isin(scales, [0x7F, 0xFF]), 16, axis=1)
+    assert ok and np.array_equal(got[finite], ref[finite])
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_pack_check_workload_weights(name):
+    packed, scales, gs = quantized(name)
+    N, K = packed.shape[0], packed.shape[1] * 2
+    got, bad, ok = pack_check(packed, scales, gs, N, K)
+    assert ok and bad == 0
+    assert np.array_equal(got, oracle.dequant_bf16_nogs(packed, scales, N, K))
+
+
+# ----- GPU quantiser (bit exact against the oracle's quantiser) ------------
+
+def gpu_quantize(W):
+    N, K = W.shape
+    wd = torch.from_numpy(np.ascontiguousarray(W, np.float32)).cuda()
+    p = torch.zeros((N, K // 2), dtype=torch.uint8, device="cuda")
+    s = torch.zeros((N, K // 16), dtype=torch.uint8, device="cuda")
+    g = torch.zeros(1, dtype=torch.float32, device="cuda")
+    bad = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_quantize(wd, N, K, p, s, g, bad)
+    torch.cuda.synchronize()
+    return p.cpu().numpy(), s.cpu().numpy(), float(g.item()), int(bad.item())
+
+
+def quantizer_cases():
+    rng = np.random.default_rng(11)
+    yield "tiny", synth.weights_f32(synth.WORKLOADS["tiny"])
+    # magnitudes spread over many binades, so scales hit subnormal and saturated codes
+    W = (np.exp2(rng.uniform(-30, 6, (64, 512))) * rng.choice([-1, 1], (64, 512))).astype(np.float32)
+    yield "logspread", W
+    W = rng.normal(0, 1, (32, 256)).astype(np.float32)
+    W[3, 16:32] = 0.0
+    W[5, :] = 0.0
+    W[7, 40] = -1e-30
+    yield "zeros", W
+    # exact E2M1 midpoints under a power-of-two scale
+    unit = 2.0 ** -8 * 2.0
+    mids = np.array([6.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.75, -1.25, -1.75,
+                     -2.5, -3.5, -5.0, 0.0])
+    W = np.zeros((2, 32), np.float32)
+    W[0, :16] = mids * unit
+    W[0, 16] = 6.0 * 448.0 * 2.0 ** -8
+    W[1, :16] = -mids * unit
+    yield "ties", W
+
+
+@pytest.mark.parametrize("case", list(range(4)))
+def test_quantizer_bit_exact(case):
+    name, W = list(quantizer_cases())[case]
+    p, s, g, bad = gpu_quantize(W)
+    rp, rs, rg = oracle.quantize(W)
+    assert bad == 0
+    assert g == rg, name
+    assert np.array_equal(s, rs), name
+    assert np.array_equal(p, rp), name
+
+
+def test_quantizer_bit_exact_decode_weights():
+    W = synth.weights_f32(synth.WORKLOADS["decode"])
+    p, s, g, bad = gpu_quantize(W)
+    rp, rs, rg = quantized("decode")
+    assert bad == 0 and g == rg
+    assert np.array_equal(s, rs)
+    assert np.array_equal(p, rp)
+
+
+def test_quantizer_flags_nonfinite():
+    W = np.zeros((2, 32), np.float32)
+    W[0, 3] = np.nan
+    W[1, 5] = np.inf
+    _, _, _, bad = gpu_quantize(W)
+    assert bad == 2
+
+
+# ----- the linear ----------------------------------------------------------
+
+def tiny_weights():
+    return Weights(*quantized("tiny"))
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 8, 12, 16])
+def test_linear_tiny_all_variants(M):
+    w = tiny_weights()
+    X = synth.x_bf16_custom(synth.X_NORMAL, M, w.K, seed=M)
+    y_ref, ad = oracle.linear(w.packed_h, w.scales_h, w.gs, X, M, w.N, w.K)
+    for v in variants_for(M, w.N, w.K):
+        y, ok, info = run_linear(w, X, v)
+        assert ok, ("guard bytes overwritten", VNAME[v])
+        check_tolerance(y, y_ref, ad)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 520, 512), (3, 1000, 768), (5, 129, 256), (16, 777, 1280),
+                                   (2, 1, 256), (9, 4097, 512)])
+def test_linear_ragged_shapes(M, N, K):
+    """N not a multiple of any tile; several tiles plus a ragged tail."""
+    W = synth.normal_f32(N * K, 0.02, seed=3, stream=7).reshape(N, K)
+    packed, scales, gs = oracle.quantize(W)
+    w = Weights(packed, scales, gs)
+    X = synth.x_bf16_custom(synth.X_OUTLIERS, M, K, seed=5, n_outliers=4, gain=20.0)
+    y_ref, ad = oracle.linear(packed, scales, gs, X, M, N, K)
+    for v in variants_for(M, N, K):
+        y, ok, _ = run_linear(w, X, v)
+        assert ok, VNAME[v]
+        check_tolerance(y, y_ref, ad)
+
+
+def test_linear_one_hot_is_exact():
+    """X = e_k with gs a power of two: Y[:, n] = bf16(gs * w_hat[n][k]) exactly,
+    whatever the summation order."""
+    w0 = quantized("tiny")
+    w = Weights(w0[0], w0[1], 2.0 ** -12)
+    D = oracle.dequant_f64(w.packed_h, w.scales_h, w.gs, w.N, w.K)
+    for k in (0, 1, 31, 200, 255):
+        X = np.zeros((1, w.K), np.uint16)
+        X[0, k] = 0x3F80
+        expect = oracle.bf16_round_array(D[:, k])
+        for v in variants_for(1, w.N, w.K):
+            y, ok, _ = run_linear(w, X, v)
+            assert ok and np.array_equal(y[0], expect), (k, VNAME[v])
+
+
+def test_linear_dyadic_small_integers_exact():
+    """Small-integer X, codes cycling through all 16 values, scales 1 or 2,
+    gs = 1: every partial sum is an integer or half-integer well inside fp32's
+    exact range, so Y equals the oracle's fp64 value rounded once to bf16."""
+    M, N, K = 4, 32, 256
+    codes = np.array([[(n + k) % 16 for k in range(K)] for n in range(N)], np.uint8)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    scales = np.array([[0x38 if (n + b) % 2 == 0 else 0x40 for b in range(K // 16)]
+                       for n in range(N)], np.uint8)
+    xs = np.array([[(k % 5) - m for k in range(K)] for m in range(M)], np.float64)
+    X = oracle.bf16_round_array(xs)
+    y_ref, _ = oracle.linear(packed, scales, 1.0, X, M, N, K)
+    expect = oracle.bf16_round_array(y_ref)
+    w = Weights(packed, scales, 1.0)
+    for v in variants_for(M, N, K):
+        y, ok, _ = run_linear(w, X, v)
+        assert ok and np.array_equal(y, expect), VNAME[v]
+
+
+def test_linear_doubling_x_doubles_y_exactly():
+    w = tiny_weights()
+    X = synth.x_bf16_custom(synth.X_NORMAL, 2, w.K, seed=9)
+    X2 = (X.astype(np.uint32) + 0x80).astype(np.uint16)
+    X2[(X & 0x7FFF) == 0] = X[(X & 0x7FFF) == 0]
+    for v in variants_for(2, w.N, w.K):
+        y1, _, _ = run_linear(w, X, v)
+        y2, _, _ = run_linear(w, X2, v)
+        a = oracle.bf16_bits_to_f64(y1)
+        b = oracle.bf16_bits_to_f64(y2)
+        assert np.array_equal(2 * a, b), VNAME[v]
+
+
+def test_linear_deterministic_and_rows_independent():
+    packed, scales, gs = quantized("decode")
+    w = Weights(packed, scales, gs)
+    X = synth.x_bf16(synth.WORKLOADS["verify"], 16)
+    for v in variants_for(16, w.N, w.K):
+        y1, _, _ = run_linear(w, X, v)
+        y2, _, _ = run_linear(w, X, v, repeat=2)
+        assert np.array_equal(y1, y2), VNAME[v]
+
+
+def test_linear_k_zero_writes_zeros_and_n_zero_is_noop():
+    w = Weights(np.zeros((8, 0), np.uint8), np.zeros((8, 0), np.uint8), 1.0)
+    w.packed = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    w.scales = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    X = np.zeros((2, 0), np.uint16)
+    plan = nv.nvfp4_linear_plan(2, 8, 0, torch.cuda.current_device(), 0)
+    try:
+        y = Guarded(16)
+        xd = torch.zeros(8, dtype=torch.int16, device="cuda")
+        nv.nvfp4_linear_run(plan, w.packed, w.scales, w.gsd, xd, y.view)
+        torch.cuda.synchronize()
+        assert y.guards_intact() and int((y.view != 0).sum()) == 0
+    finally:
+        nv.nvfp4_linear_destroy(plan)
+    plan = nv.nvfp4_linear_plan(1, 0, 256, torch.cuda.current_device(), 0)
+    nv.nvfp4_linear_run(plan, None, None, w.gsd, None, w.gsd)
+    nv.nvfp4_linear_destroy(plan)
+
+
+def test_linear_argument_errors_launch_nothing():
+    w = tiny_weights()
+    plan = nv.nvfp4_linear_plan(1, w.N, w.K, torch.cuda.current_device(), 0)
+    try:
+        xd = dev(synth.x_bf16(synth.WORKLOADS["tiny"], 1))
+        y = Guarded(w.N)
+        base = w.packed.data_ptr()
+        cases = [
+            ((base + 8, w.scales, w.gsd, xd, y.view), nv.NVFP4_ERR_MISALIGNED),
+            ((w.packed, w.scales, w.gsd, xd.data_ptr() + 2, y.view), nv.NVFP4_ERR_MISALIGNED),
+            ((w.packed, None, w.gsd, xd, y.view), nv.NVFP4_ERR_INVALID_ARG),
+            ((w.packed, w.scales, None, xd, y.view), nv.NVFP4_ERR_INVALID_ARG),
+            ((w.packed, w.scales, w.gsd, xd, None), nv.NVFP4_ERR_INVALID_ARG),
+        ]
+        for args, status in cases:
+            s = nv.nvfp4_linear_run(plan, *args, check=False)
+            assert s == status
+        torch.cuda.synchronize()
+        assert int((y.view != 0x5A5A).sum()) == 0      # nothing was written
+    finally:
+        nv.nvfp4_linear_destroy(plan)
+    with pytest.raises(nv.Nvfp4Error):
+        nv.nvfp4_linear_plan(1, 8, 256, torch.cuda.device_count(), 0)
+
+
+# ----- full-size workloads ------------------------------------------------
+
+def full_check(name, M, copy=0, rows=None):
+    packed, scales, gs = quantized(name, copy)
+    w = Weights(packed, scales, gs)
+    wl = synth.WORKLOADS[name]
+    X = synth.x_bf16(wl, M)
+    results = {}
+    for v in variants_for(M, w.N, w.K):
+        y, ok, info = run_linear(w, X, v)
+        assert ok, VNAME[v]
+        results[v] = y
+    if rows is None:
+        y_ref, ad = oracle.linear(packed, scales, gs, X, M, w.N, w.K)
+        for v, y in results.items():
+            check_tolerance(y, y_ref, ad)
+    else:
+        y_ref, ad = oracle.linear(packed, scales, gs, X, M, w.N, w.K, rows=rows)
+        for v, y in results.items():
+            check_tolerance(y[:, rows], y_ref, ad)
+    return results
+
+
+def test_decode_projection_full():
+    full_check("decode", 1)
+
+
+@pytest.mark.parametrize("M", [2, 4, 8, 12, 16])
+def test_verify_projection_full(M):
+    full_check("verify", M)
+
+
+@pytest.mark.parametrize("M", [1, 4, 8, 16])
+def test_down_projection_full(M):
+    full_check("down", M)
