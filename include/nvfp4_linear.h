@@ -93,10 +93,12 @@ typedef struct nvfp4_plan_s* nvfp4_plan_t;
 nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
                                nvfp4_plan_t* out);
 
-/* Device workspace bytes nvfp4_linear_run needs for this plan (split-K
- * partials, tile counters and the 4-byte status word), 0 if none. The
- * workspace must be zero-filled once before its first use; the kernels leave
- * it zero-filled again after every run. */
+/* Device workspace bytes nvfp4_linear_run needs for this plan (status word,
+ * per-tile counters and fp32 partials of tiles computed in several pieces),
+ * 0 if none. Zero-fill it once before first use: after every successful run
+ * its status word and counters are zero again, so it can be reused without
+ * clearing (the partial area never needs clearing). Two runs in flight at the
+ * same time must not share a workspace. */
 size_t nvfp4_linear_workspace_bytes(nvfp4_plan_t plan);
 
 /* Chosen variant (NVFP4_VARIANT_*) and split-K factor of a plan; -1 if null. */

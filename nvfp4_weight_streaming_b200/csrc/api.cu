@@ -6,10 +6,22 @@
 #include "nvfp4_linear.h"
 #include "kernels.h"
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 #include <cstdlib>
+#include <mutex>
 #include <new>
+
+namespace {
+// TMA descriptors of one weight set, keyed by its two device pointers.
+struct MapEntry {
+  const void* wp = nullptr;
+  const void* ws = nullptr;
+  CUtensorMap mw, ms;
+};
+constexpr int kMapCache = 16;
+}  // namespace
 
 struct nvfp4_plan_s {
   int M, N, K, device;
@@ -19,6 +31,10 @@ struct nvfp4_plan_s {
   int num_sms;
   size_t ws_bytes;
   nvfp4::GemvConfig gemv;
+  nvfp4::TcConfig tc;
+  std::mutex map_mu;
+  MapEntry maps[kMapCache];
+  int map_next = 0;
 };
 
 namespace {
@@ -34,10 +50,36 @@ nvfp4_status check_device(int device) {
 // Which variant AUTO takes for a shape: the fastest measured on B200 for
 // that (M, N, K) class among those that can run it.
 int auto_variant(int M, int N, int K) {
-  (void)N;
-  if (M <= 4 && size_t(M) * size_t(K) * 4 <= 200 * 1024) return int(NVFP4_VARIANT_GEMV);
-  return int(NVFP4_VARIANT_GEMV);
+  (void)M; (void)N; (void)K;
+  return int(NVFP4_VARIANT_TC);
 }
+
+// Copy of the TMA descriptors for (wp, ws), encoding them on first use.
+bool lookup_maps(nvfp4_plan_s* p, const void* wp, const void* ws, CUtensorMap* mw, CUtensorMap* ms) {
+  std::lock_guard<std::mutex> g(p->map_mu);
+  for (int i = 0; i < kMapCache; ++i) {
+    if (p->maps[i].wp == wp && p->maps[i].ws == ws) {
+      *mw = p->maps[i].mw;
+      *ms = p->maps[i].ms;
+      return true;
+    }
+  }
+  MapEntry& e = p->maps[p->map_next];
+  if (!nvfp4::tc_encode_maps(p->tc, static_cast<const uint8_t*>(wp),
+                             static_cast<const uint8_t*>(ws), &e.mw, &e.ms)) {
+    e.wp = e.ws = nullptr;
+    return false;
+  }
+  e.wp = wp;
+  e.ws = ws;
+  p->map_next = (p->map_next + 1) % kMapCache;
+  *mw = e.mw;
+  *ms = e.ms;
+  return true;
+}
+
+constexpr long long kTimeoutCycles = 1ll << 31;       // ~1 s at 2 GHz
+constexpr long long kStallTimeoutCycles = 1ll << 22;  // test mode: ~2 ms
 
 }  // namespace
 
@@ -72,12 +114,18 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   if (cudaGetDevice(&prev) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (prev != device && cudaSetDevice(device) != cudaSuccess) return NVFP4_ERR_CUDA;
 
-  nvfp4_plan_s p{};
+  nvfp4_plan_s* h = new (std::nothrow) nvfp4_plan_s();
+  if (!h) { if (prev != device) cudaSetDevice(prev); return NVFP4_ERR_CUDA; }
+  nvfp4_plan_s& p = *h;
   p.M = M; p.N = N; p.K = K; p.device = device; p.flags = flags; p.num_sms = sms;
   p.split_k = 1;
   p.ws_bytes = 0;
   unsigned forced = flags & NVFP4_PLAN_VARIANT_MASK;
   p.variant = forced ? int(forced) : auto_variant(M, N, K);
+  if (K == 0 || N == 0) {
+    // nothing to contract: run() writes zeros (K == 0) or returns (N == 0)
+    if (p.variant == int(NVFP4_VARIANT_GEMV) && M > 4) p.variant = int(NVFP4_VARIANT_TC);
+  }
   nvfp4_status st = NVFP4_OK;
   switch (p.variant) {
     case NVFP4_VARIANT_GEMV: {
@@ -86,13 +134,21 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
       if (K > 0 && N > 0 && nvfp4::gemv_configure(p.gemv, sms) != cudaSuccess) st = NVFP4_ERR_CUDA;
       break;
     }
+    case NVFP4_VARIANT_TC: {
+      if (K == 0 || N == 0) break;
+      p.tc.M = M; p.tc.N = N; p.tc.K = K;
+      cudaError_t e = nvfp4::tc_configure(p.tc, sms);
+      if (e == cudaErrorNotSupported || e == cudaErrorInvalidConfiguration) st = NVFP4_ERR_UNSUPPORTED;
+      else if (e != cudaSuccess) st = NVFP4_ERR_CUDA;
+      p.split_k = p.tc.S;
+      p.ws_bytes = p.tc.ws_bytes;
+      break;
+    }
     default:
       st = NVFP4_ERR_UNSUPPORTED;
   }
   if (prev != device) cudaSetDevice(prev);
-  if (st != NVFP4_OK) return st;
-  nvfp4_plan_s* h = new (std::nothrow) nvfp4_plan_s(p);
-  if (!h) return NVFP4_ERR_CUDA;
+  if (st != NVFP4_OK) { delete h; return st; }
   *out = h;
   return NVFP4_OK;
 }
@@ -132,6 +188,14 @@ nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
       case NVFP4_VARIANT_GEMV:
         e = nvfp4::launch_gemv(plan->gemv, w_packed, w_scales, w_global, xb, yb, st);
         break;
+      case NVFP4_VARIANT_TC: {
+        CUtensorMap mw, ms;
+        if (!lookup_maps(plan, w_packed, w_scales, &mw, &ms)) return NVFP4_ERR_CUDA;
+        const bool stall = (plan->flags & NVFP4_PLAN_TEST_STALL) != 0;
+        e = nvfp4::launch_tc(plan->tc, &mw, &ms, w_global, xb, yb, workspace,
+                             stall ? kStallTimeoutCycles : kTimeoutCycles, stall, st);
+        break;
+      }
       default:
         return NVFP4_ERR_UNSUPPORTED;
     }
@@ -149,9 +213,9 @@ nvfp4_status nvfp4_linear_status(nvfp4_plan_t plan, void* workspace, void* strea
     if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
       return NVFP4_ERR_CUDA;
     if (word != 0) {
-      uint32_t zero = 0;
-      if (cudaMemcpy(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
-        return NVFP4_ERR_CUDA;
+      // an aborted run can leave split counters behind: clear the whole workspace
+      if (cudaMemset(workspace, 0, plan->ws_bytes) != cudaSuccess) return NVFP4_ERR_CUDA;
+      if (cudaDeviceSynchronize() != cudaSuccess) return NVFP4_ERR_CUDA;
       return NVFP4_ERR_TIMEOUT;
     }
   }

@@ -106,8 +106,13 @@ cudaError_t launch_m(const GemvConfig& c, const uint8_t* wp, const uint8_t* ws, 
 
 template <int M>
 cudaError_t config_m(GemvConfig& c, int num_sms) {
-  cudaError_t e = cudaFuncSetAttribute(k_gemv<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(c.smem));
+  // per-function attribute shared by all plans: raise it to the opt-in maximum
+  int dev = 0, optin = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  if (c.smem > size_t(optin)) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(k_gemv<M>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_gemv<M>, c.block, c.smem);

@@ -30,4 +30,19 @@ cudaError_t gemv_configure(GemvConfig& c, int num_sms);
 cudaError_t launch_gemv(const GemvConfig& c, const uint8_t* wp, const uint8_t* ws,
                         const float* gs, const uint16_t* x, uint16_t* y, cudaStream_t st);
 
+// tcgen05 tensor-core variant (k_tc.cu).
+struct TcConfig {
+  int M, N, K;
+  int tiles, S, P, ks_base, ks_rem, nb, xk_max, pmax, grid;
+  bool split;
+  size_t smem, ws_counters_off, ws_partials_off, ws_bytes;
+};
+cudaError_t tc_configure(TcConfig& c, int num_sms);
+// Encode the TMA descriptors (CUtensorMap, 128 bytes each) for one weight set.
+bool tc_encode_maps(const TcConfig& c, const uint8_t* wp, const uint8_t* ws, void* map_w,
+                    void* map_s);
+cudaError_t launch_tc(const TcConfig& c, const void* map_w, const void* map_s, const float* gs,
+                      const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
+                      bool stall, cudaStream_t st);
+
 }  // namespace nvfp4
