@@ -132,24 +132,33 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(world, value: float) -> float:
+def _reduce(world, value: float, op) -> float:
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    device = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(world, value: float) -> float:
+    """Timing across replicas: the slowest rank defines the step time."""
+    import torch.distributed as dist
+    return _reduce(world, value, dist.ReduceOp.MAX if world > 1 else None)
 
 
 def sum_over_ranks(world, value: float) -> float:
-    if world == 1:
-        return value
-    import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(world, value, dist.ReduceOp.SUM if world > 1 else None)
+
+
+def aggregate(world: int, bytes_per_call: float, sec_per_call_this_rank: float):
+    """(seconds per call = max over ranks, whole-job GB/s = all ranks' bytes / that time)."""
+    sec = max_over_ranks(world, sec_per_call_this_rank)
+    total_bytes = sum_over_ranks(world, bytes_per_call)
+    return sec, effective_gbs(total_bytes, sec)
 
 
 # ---------------------------------------------------------------------------

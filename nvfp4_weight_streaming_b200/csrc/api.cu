@@ -32,6 +32,7 @@ struct nvfp4_plan_s {
   size_t ws_bytes;
   nvfp4::GemvConfig gemv;
   nvfp4::TcConfig tc;
+  nvfp4::MmaConfig mma;
   std::mutex map_mu;
   MapEntry maps[kMapCache];
   int map_next = 0;
@@ -49,8 +50,13 @@ nvfp4_status check_device(int device) {
 
 // Which variant AUTO takes for a shape: the fastest measured on B200 for
 // that (M, N, K) class among those that can run it.
+// Measured on B200 for the 5120 x 34816 projection: the CUDA-core GEMV is
+// fastest at M = 1, the mma.sync pipeline up to M = 8, the tcgen05 pipeline
+// beyond (its MMA cost does not grow with the token count).
 int auto_variant(int M, int N, int K) {
-  (void)M; (void)N; (void)K;
+  (void)N;
+  if (M == 1 && size_t(K) * 4 <= 200 * 1024) return int(NVFP4_VARIANT_GEMV);
+  if (M <= 8) return int(NVFP4_VARIANT_MMA);
   return int(NVFP4_VARIANT_TC);
 }
 
@@ -65,8 +71,9 @@ bool lookup_maps(nvfp4_plan_s* p, const void* wp, const void* ws, CUtensorMap* m
     }
   }
   MapEntry& e = p->maps[p->map_next];
-  if (!nvfp4::tc_encode_maps(p->tc, static_cast<const uint8_t*>(wp),
-                             static_cast<const uint8_t*>(ws), &e.mw, &e.ms)) {
+  const int box_rows = p->variant == int(NVFP4_VARIANT_MMA) ? nvfp4::kMmaTileRows : 128;
+  if (!nvfp4::encode_weight_maps(p->N, p->K, box_rows, static_cast<const uint8_t*>(wp),
+                                 static_cast<const uint8_t*>(ws), &e.mw, &e.ms)) {
     e.wp = e.ws = nullptr;
     return false;
   }
@@ -126,26 +133,48 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
     // nothing to contract: run() writes zeros (K == 0) or returns (N == 0)
     if (p.variant == int(NVFP4_VARIANT_GEMV) && M > 4) p.variant = int(NVFP4_VARIANT_TC);
   }
-  nvfp4_status st = NVFP4_OK;
-  switch (p.variant) {
-    case NVFP4_VARIANT_GEMV: {
-      if (M > 4 || size_t(M) * size_t(K) * 4 > 200 * 1024) { st = NVFP4_ERR_UNSUPPORTED; break; }
-      p.gemv.M = M; p.gemv.N = N; p.gemv.K = K;
-      if (K > 0 && N > 0 && nvfp4::gemv_configure(p.gemv, sms) != cudaSuccess) st = NVFP4_ERR_CUDA;
-      break;
+  auto configure = [&]() -> nvfp4_status {
+    nvfp4_status st = NVFP4_OK;
+    switch (p.variant) {
+      case NVFP4_VARIANT_GEMV: {
+        if (M > 4 || size_t(M) * size_t(K) * 4 > 200 * 1024) { st = NVFP4_ERR_UNSUPPORTED; break; }
+        p.gemv.M = M; p.gemv.N = N; p.gemv.K = K;
+        if (K > 0 && N > 0 && nvfp4::gemv_configure(p.gemv, sms) != cudaSuccess) st = NVFP4_ERR_CUDA;
+        break;
+      }
+      case NVFP4_VARIANT_MMA: {
+        if (K == 0 || N == 0) break;
+        p.mma.M = M; p.mma.N = N; p.mma.K = K;
+        cudaError_t e = nvfp4::mma_configure(p.mma, sms);
+        if (e == cudaSuccess && !nvfp4::tensor_maps_supported()) e = cudaErrorNotSupported;
+        if (e == cudaErrorInvalidConfiguration || e == cudaErrorNotSupported) st = NVFP4_ERR_UNSUPPORTED;
+        else if (e != cudaSuccess) st = NVFP4_ERR_CUDA;
+        p.split_k = p.mma.S;
+        p.ws_bytes = p.mma.ws_bytes;
+        break;
+      }
+      case NVFP4_VARIANT_TC: {
+        if (K == 0 || N == 0) break;
+        p.tc.M = M; p.tc.N = N; p.tc.K = K;
+        cudaError_t e = nvfp4::tc_configure(p.tc, sms);
+        if (e == cudaErrorNotSupported || e == cudaErrorInvalidConfiguration) st = NVFP4_ERR_UNSUPPORTED;
+        else if (e != cudaSuccess) st = NVFP4_ERR_CUDA;
+        p.split_k = p.tc.S;
+        p.ws_bytes = p.tc.ws_bytes;
+        break;
+      }
+      default:
+        st = NVFP4_ERR_UNSUPPORTED;
     }
-    case NVFP4_VARIANT_TC: {
-      if (K == 0 || N == 0) break;
-      p.tc.M = M; p.tc.N = N; p.tc.K = K;
-      cudaError_t e = nvfp4::tc_configure(p.tc, sms);
-      if (e == cudaErrorNotSupported || e == cudaErrorInvalidConfiguration) st = NVFP4_ERR_UNSUPPORTED;
-      else if (e != cudaSuccess) st = NVFP4_ERR_CUDA;
-      p.split_k = p.tc.S;
-      p.ws_bytes = p.tc.ws_bytes;
-      break;
-    }
-    default:
-      st = NVFP4_ERR_UNSUPPORTED;
+    return st;
+  };
+  nvfp4_status st = configure();
+  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.variant != int(NVFP4_VARIANT_TC)) {
+    // the automatic choice cannot take this shape: the tcgen05 pipeline can
+    p.variant = int(NVFP4_VARIANT_TC);
+    p.split_k = 1;
+    p.ws_bytes = 0;
+    st = configure();
   }
   if (prev != device) cudaSetDevice(prev);
   if (st != NVFP4_OK) { delete h; return st; }
@@ -188,6 +217,14 @@ nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
       case NVFP4_VARIANT_GEMV:
         e = nvfp4::launch_gemv(plan->gemv, w_packed, w_scales, w_global, xb, yb, st);
         break;
+      case NVFP4_VARIANT_MMA: {
+        CUtensorMap mw, ms;
+        if (!lookup_maps(plan, w_packed, w_scales, &mw, &ms)) return NVFP4_ERR_CUDA;
+        const bool stall = (plan->flags & NVFP4_PLAN_TEST_STALL) != 0;
+        e = nvfp4::launch_mma(plan->mma, &mw, &ms, w_global, xb, yb, workspace,
+                              stall ? kStallTimeoutCycles : kTimeoutCycles, stall, st);
+        break;
+      }
       case NVFP4_VARIANT_TC: {
         CUtensorMap mw, ms;
         if (!lookup_maps(plan, w_packed, w_scales, &mw, &ms)) return NVFP4_ERR_CUDA;

@@ -58,7 +58,11 @@ constexpr int W_BYTES = ROWS * KC / 2;   // 16384
 constexpr int S_BYTES = ROWS * KC / 16;  // 2048
 constexpr int A_COLS = KC / 2;           // TMEM columns per A stage (two f16 per column)
 constexpr int D_COL0 = TSTAGE * A_COLS;  // 384: first accumulator column
-constexpr int D_COLS = 32;               // columns per accumulator buffer
+constexpr int D_COLS = 64;               // columns per accumulator buffer (2 buffers)
+// Consecutive MMAs of a stage rotate over D_COLS / n_mma independent
+// accumulators (4 at N = 16, 2 at N = 32): MMAs into one accumulator
+// serialise on it, independent ones overlap. The epilogue adds them.
+
 constexpr int TMEM_COLS = 512;
 constexpr int NUM_WARPS = 14;
 constexpr int NUM_THREADS = NUM_WARPS * 32;
@@ -105,50 +109,8 @@ __host__ __device__ inline Smem smem_layout(int nb, int xk_max) {
 
 // ---- PTX wrappers ---------------------------------------------------------
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(b) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_test(uint32_t b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok) : "r"(b), "r"(parity) : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* tm, int x, int y,
-                                            uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-      ::"r"(dst), "l"(tm), "r"(x), "r"(y), "r"(bar) : "memory");
-}
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void named_bar(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-// bar.red.and over `count` threads: every participant gets the AND of `ok`.
-__device__ __forceinline__ bool named_bar_and(int id, int count, bool ok) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.b32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r) : "r"(ok ? 1u : 0u), "r"(id), "r"(count) : "memory");
-  return r != 0;
-}
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
   // K-major, no swizzle: 8-row x 16-byte core matrices; lbo = byte step
   // between the two 16-byte K halves of an MMA, sbo = byte step between
@@ -232,17 +194,6 @@ __device__ __forceinline__ Slice my_slice(const Params& p) {
   return q;
 }
 
-// Number of CTA boundaries floor(c*L/P), c in [1, P), with lo < boundary <= hi.
-__device__ __forceinline__ long long boundaries_in(long long lo, long long hi, long long L, int P) {
-  if (hi <= lo) return 0;
-  // c >= ceil((lo+1)*P/L)  and  c <= ceil((hi+1)*P/L) - 1
-  long long cmin = ((lo + 1) * P + L - 1) / L;
-  long long cmax = ((hi + 1) * P + L - 1) / L - 1;
-  if (cmin < 1) cmin = 1;
-  if (cmax > P - 1) cmax = P - 1;
-  return cmax >= cmin ? cmax - cmin + 1 : 0;
-}
-
 __device__ __forceinline__ int slice_cnt(const Params& p, int s) {
   return p.ks_base + (s < p.ks_rem ? 1 : 0);
 }
@@ -255,21 +206,6 @@ __device__ __forceinline__ int pieces_in_slice(const Params& p, int t, int s) {
 }
 
 // ---- X staging helpers ----------------------------------------------------
-
-// Exponent of a nonzero finite bf16 value, and its 8-bit significand (128..255).
-__device__ __forceinline__ int bf16_exp(uint32_t b, uint32_t& sig) {
-  const uint32_t e8 = (b >> 7) & 0xFFu, mant = b & 0x7Fu;
-  if (e8) { sig = 0x80u | mant; return int(e8) - 127; }
-  const int msb = 31 - __clz(int(mant));
-  sig = mant << (7 - msb);
-  return msb - 133;
-}
-
-// f16 bits of sign * sig/128 * 2^t for a normal f16 exponent t (else 0).
-__device__ __forceinline__ uint32_t make_f16(uint32_t sign, int t, uint32_t sig) {
-  if (t < -14 || t > 15) return 0;
-  return (sign << 15) | (uint32_t(t + 15) << 10) | ((sig & 0x7Fu) << 3);
-}
 
 // ---- the kernel -------------------------------------------------------------
 
@@ -344,52 +280,76 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
           drain_bar(b_full + 8 * int(i % NSTAGE), uint32_t(i / NSTAGE) & 1u, p);
       }
     }
+    __syncwarp();   // lanes 1..31 wait here for lane 0 before the block barrier
   } else {
     // -------------------------------------------- stage X (warps 2..13)
     if (warp >= WARP_DEC0) {
+      // Every chunk (8 consecutive k of one token) is loaded once, all loads
+      // of a thread in flight together; the slice holds at most
+      // (nb/2) * xk_max / 8 <= 8 * 384 chunks, i.e. <= 8 per thread.
+      constexpr int MAXC = 8;
       const int ts = threadIdx.x - WARP_DEC0 * 32, nts = (NUM_WARPS - WARP_DEC0) * 32;
       const int chunks = klen / 8;
-      for (int u = ts; u < p.M * chunks; u += nts) {
-        const int m = u / chunks, kc = u - m * chunks;
-        const uint4 v = *reinterpret_cast<const uint4*>(p.x + size_t(m) * p.K + k0e + 8 * kc);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        int mx = INT_MIN;
+      const int nreal = p.M * chunks;
+      uint4 xv[MAXC];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t b = (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
-          if (b & 0x7FFFu) { uint32_t sg; mx = max(mx, bf16_exp(b, sg)); }
+      for (int c = 0; c < MAXC; ++c) {
+        const int u = ts + c * nts;
+        if (u < nreal) {
+          const int m = u / chunks, kc = u - m * chunks;
+          xv[c] = *reinterpret_cast<const uint4*>(p.x + size_t(m) * p.K + k0e + 8 * kc);
         }
-        if (mx != INT_MIN) atomicMax(&emax[m], mx);
+      }
+#pragma unroll
+      for (int c = 0; c < MAXC; ++c) {
+        const int u = ts + c * nts;
+        if (u < nreal) {
+          const int m = u / chunks;
+          const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+          int mx = INT_MIN;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t b = (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
+            if (b & 0x7FFFu) { uint32_t sg; mx = max(mx, bf16_exp(b, sg)); }
+          }
+          if (mx != INT_MIN) atomicMax(&emax[m], mx);
+        }
       }
       named_bar(BAR_STAGERS, (NUM_WARPS - WARP_DEC0) * 32);
       const int mrows = p.M <= 8 ? 8 : 16;       // rows per plane
       bool lo_used = false;
-      for (int u = ts; u < p.nb * chunks; u += nts) {
-        const int r = u / chunks, kc = u - r * chunks;
-        const int m = r % mrows;
-        const bool lo_plane = r >= mrows;
-        uint32_t o[4] = {0u, 0u, 0u, 0u};
-        if (m < p.M && emax[m] != INT_MIN) {
-          const int sh = 14 - emax[m];
-          const uint4 v = *reinterpret_cast<const uint4*>(p.x + size_t(m) * p.K + k0e + 8 * kc);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int c = 0; c < MAXC; ++c) {
+        const int u = ts + c * nts;
+        if (u < nreal) {
+          const int m = u / chunks, kc = u - m * chunks;
+          const int sh = (emax[m] == INT_MIN) ? 0 : 14 - emax[m];
+          const uint32_t w[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
+          uint32_t hi[4] = {0u, 0u, 0u, 0u}, lo[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const uint32_t b = (w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;
-            uint32_t h = 0;
             if (b & 0x7FFFu) {
               uint32_t sg;
-              const int e = bf16_exp(b, sg);
-              const int th = e + sh;
-              if (!lo_plane) h = (th >= -14) ? make_f16(b >> 15, th, sg) : 0u;
-              else h = (th >= -14) ? 0u : make_f16(b >> 15, th + LO_SHIFT, sg);
+              const int th = bf16_exp(b, sg) + sh;
+              if (th >= -14) hi[i >> 1] |= make_f16(b >> 15, th, sg) << (16 * (i & 1));
+              else lo[i >> 1] |= make_f16(b >> 15, th + LO_SHIFT, sg) << (16 * (i & 1));
             }
-            o[i >> 1] |= h << (16 * (i & 1));
           }
-          if (lo_plane && (o[0] | o[1] | o[2] | o[3])) lo_used = true;
+          lo_used |= (lo[0] | lo[1] | lo[2] | lo[3]) != 0u;
+          const int rl = mrows + m;
+          *reinterpret_cast<uint4*>(sX + kc * 128 + (m >> 3) * sbo + (m & 7) * 16) =
+              make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(sX + kc * 128 + (rl >> 3) * sbo + (rl & 7) * 16) =
+              make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
-        *reinterpret_cast<uint4*>(sX + kc * 128 + (r >> 3) * sbo + (r & 7) * 16) =
-            make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      // rows of tokens >= M (both planes) are zero
+      const int npad = mrows - p.M;
+      for (int u = ts; u < 2 * npad * chunks; u += nts) {
+        const int pr = u / chunks, kc = u - pr * chunks;
+        const int r = (pr < npad) ? (p.M + pr) : (mrows + p.M + pr - npad);
+        *reinterpret_cast<uint4*>(sX + kc * 128 + (r >> 3) * sbo + (r & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
       }
       if (lo_used) atomicOr(&misc[2], 1u);
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -398,6 +358,7 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
     fence_after();
     const bool need_lo = misc[2] != 0;
     const int n_mma = (p.M <= 8) ? 16 : (need_lo ? 32 : 16);
+    const int nacc = D_COLS / n_mma;
 
     if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
@@ -427,7 +388,8 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
             for (int kk = 0; kk < KC / 16; ++kk) {
               const uint32_t a_tmem = tmem + ts * A_COLS + kk * 8;
               const uint64_t bd = smem_desc(x_base + uint32_t(j * KC + kk * 16) * 16u, 128u, sbo);
-              mma_f16_ts(d_tmem, a_tmem, bd, idesc, (first && kk == 0) ? 0u : 1u);
+              const int acc_i = kk % nacc;
+              mma_f16_ts(d_tmem + acc_i * n_mma, a_tmem, bd, idesc, (first && kk < nacc) ? 0u : 1u);
             }
             first = false;
             mma_commit(b_aempty + 8 * ts);
@@ -440,6 +402,7 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
         mma_commit(b_done);
         drain_bar(b_done, 0u, p);
       }
+      __syncwarp();   // reconverge warp 1 before the block barrier and dealloc
     } else if (warp < WARP_EPI0) {
       // ------------------------------------------------------------ decoders
       const int q = warp & 3, h = (warp - WARP_DEC0) >> 2;
@@ -493,6 +456,15 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
       const float gs = *p.gs;
       const int et = threadIdx.x - WARP_EPI0 * 32;          // 0..127
       const int mrows = p.M <= 8 ? 8 : 16;
+      // unscale factors of the hi and lo planes per token (exact powers of two)
+      float f_hi[16], f_lo[16];
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        const bool live = m < p.M && emax[m] != INT_MIN;
+        const int sh = live ? 14 - emax[m] : 0;
+        f_hi[m] = live ? ldexpf(1.0f, -sh) : 0.0f;
+        f_lo[m] = (live && mrows + m < n_mma) ? ldexpf(1.0f, -(sh + LO_SHIFT)) : 0.0f;
+      }
       int sidx = 0;
       long long idx = sl.a;
       while (idx < sl.b) {
@@ -505,11 +477,24 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
                                  ST_TIMEOUT_EPI);
         if (!named_bar_and(BAR_EPI, NUM_EPI * 32, ok)) break;
         fence_after();
-        uint32_t acc[32];
+        uint32_t raw[64];
         const uint32_t taddr = tmem + (uint32_t(32 * q) << 16) + D_COL0 + db * D_COLS;
-        tmem_ld16(taddr, acc);
-        if (n_mma > 16) tmem_ld16(taddr + 16, acc + 16);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (16 * u < nacc * n_mma) tmem_ld16(taddr + 16 * u, raw + 16 * u);
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        float acc[32];
+        if (n_mma == 16) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            acc[c] = ((__uint_as_float(raw[c]) + __uint_as_float(raw[16 + c])) +
+                      __uint_as_float(raw[32 + c])) + __uint_as_float(raw[48 + c]);
+            acc[16 + c] = 0.0f;
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) acc[c] = __uint_as_float(raw[c]) + __uint_as_float(raw[32 + c]);
+        }
         fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(b_dempty + 8 * db);
@@ -517,37 +502,39 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
         float v[16];
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
-          v[m] = 0.0f;
-          if (m < p.M && emax[m] != INT_MIN) {
-            const int sh = 14 - emax[m];
-            float hi = __uint_as_float(acc[m]);
-            float lo = (mrows + m < n_mma) ? __uint_as_float(acc[mrows + m]) : 0.0f;
-            v[m] = ldexpf(hi, -sh) + ldexpf(lo, -(sh + LO_SHIFT));
-          }
+          const float lo = (mrows == 8) ? acc[(8 + m) & 31] : acc[(16 + m) & 31];
+          v[m] = acc[m] * f_hi[m] + lo * f_lo[m];
         }
         // pieces of this tile: over all slices, and this piece's ordinal
         int npieces = 0;
         for (int s2 = 0; s2 < p.S; ++s2) npieces += pieces_in_slice(p, t, s2);
         const int row = t * ROWS + r;
         if (npieces == 1) {
-          if (row < p.N)
-            for (int m = 0; m < p.M; ++m) p.y[size_t(m) * p.N + row] = float_to_bf16_bits(gs * v[m]);
+          if (row < p.N) {
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+              if (m < p.M) p.y[size_t(m) * p.N + row] = float_to_bf16_bits(gs * v[m]);
+          }
           continue;
         }
         const int ord = int(boundaries_in((long long)t * sl.cnt, seg_start, sl.L, p.P));
         const long long slot = ((long long)t * p.S + sl.s) * p.pmax + ord;
         float* part = p.partials + slot * p.M * ROWS;
-        for (int m = 0; m < p.M; ++m) part[m * ROWS + r] = v[m];
-        __threadfence();
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+          if (m < p.M) part[m * ROWS + r] = v[m];
+        // publish: CTA barrier, then one gpu-scope fence + counter increment
+        // (the fence is cumulative over the writes ordered before it by the barrier)
         named_bar(BAR_EPI, NUM_EPI * 32);
         if (et == 0) {
+          __threadfence();
           const unsigned old = atomicAdd(&p.counters[t], 1u);
+          __threadfence();
           misc[3] = (old == unsigned(npieces - 1)) ? 1u : 0u;
         }
         named_bar(BAR_EPI, NUM_EPI * 32);
         const bool last = misc[3] != 0;
         if (last) {
-          __threadfence();
           float sum[16];
 #pragma unroll
           for (int m = 0; m < 16; ++m) sum[m] = 0.0f;
@@ -555,11 +542,16 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
             const int np = pieces_in_slice(p, t, s2);
             for (int o = 0; o < np; ++o) {
               const float* pp = p.partials + (((long long)t * p.S + s2) * p.pmax + o) * p.M * ROWS;
-              for (int m = 0; m < p.M; ++m) sum[m] += __ldcg(pp + m * ROWS + r);
+#pragma unroll
+              for (int m = 0; m < 16; ++m)
+                if (m < p.M) sum[m] += __ldcg(pp + m * ROWS + r);
             }
           }
-          if (row < p.N)
-            for (int m = 0; m < p.M; ++m) p.y[size_t(m) * p.N + row] = float_to_bf16_bits(gs * sum[m]);
+          if (row < p.N) {
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+              if (m < p.M) p.y[size_t(m) * p.N + row] = float_to_bf16_bits(gs * sum[m]);
+          }
           if (et == 0) atomicExch(&p.counters[t], 0u);
         }
         named_bar(BAR_EPI, NUM_EPI * 32);
@@ -609,6 +601,8 @@ cudaError_t tc_configure(TcConfig& c, int num_sms) {
   c.S = S; c.P = P; c.ks_base = ks_base; c.ks_rem = ks_rem;
   c.grid = S * P;
   c.xk_max = (ks_base + (ks_rem ? 1 : 0)) * KC;
+  // X staging holds at most 8 chunks of 8 elements per staging thread
+  if ((long long)c.M * c.xk_max / 8 > 8LL * (NUM_WARPS - WARP_DEC0) * 32) return cudaErrorInvalidConfiguration;
   // pieces per (tile, slice): simulate the boundaries
   int pmax = 1;
   bool split = S > 1;
@@ -645,29 +639,32 @@ cudaError_t tc_configure(TcConfig& c, int num_sms) {
   return cudaSuccess;
 }
 
-bool tc_encode_maps(const TcConfig& c, const uint8_t* wp, const uint8_t* ws, void* map_w,
-                    void* map_s) {
-  using namespace tc;
-  auto fn = encode_fn();
+bool encode_weight_maps(int N, int K, int box_rows, const uint8_t* wp, const uint8_t* ws,
+                        void* map_w, void* map_s) {
+  auto fn = tc::encode_fn();
   if (!fn) return false;
-  const cuuint64_t dim_w[2] = {cuuint64_t(c.K / 2), cuuint64_t(c.N)};
-  const cuuint64_t str_w[1] = {cuuint64_t(c.K / 2)};
-  const cuuint32_t box_w[2] = {KC / 2, ROWS};
+  // codes: [N][K/2] bytes, box 128 bytes x box_rows rows, 128-byte swizzle
+  const cuuint64_t dim_w[2] = {cuuint64_t(K / 2), cuuint64_t(N)};
+  const cuuint64_t str_w[1] = {cuuint64_t(K / 2)};
+  const cuuint32_t box_w[2] = {128, cuuint32_t(box_rows)};
   const cuuint32_t one[2] = {1, 1};
   CUresult r = fn(static_cast<CUtensorMap*>(map_w), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                   const_cast<uint8_t*>(wp), dim_w, str_w, box_w, one,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return false;
-  const cuuint64_t dim_s[2] = {cuuint64_t(c.K / 16), cuuint64_t(c.N)};
-  const cuuint64_t str_s[1] = {cuuint64_t(c.K / 16)};
-  const cuuint32_t box_s[2] = {KC / 16, ROWS};
+  // scales: [N][K/16] bytes, box 16 bytes x box_rows rows
+  const cuuint64_t dim_s[2] = {cuuint64_t(K / 16), cuuint64_t(N)};
+  const cuuint64_t str_s[1] = {cuuint64_t(K / 16)};
+  const cuuint32_t box_s[2] = {16, cuuint32_t(box_rows)};
   r = fn(static_cast<CUtensorMap*>(map_s), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
          const_cast<uint8_t*>(ws), dim_s, str_s, box_s, one, CU_TENSOR_MAP_INTERLEAVE_NONE,
          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+bool tensor_maps_supported() { return tc::encode_fn() != nullptr; }
 
 cudaError_t launch_tc(const TcConfig& c, const void* map_w, const void* map_s, const float* gs,
                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,

@@ -38,11 +38,27 @@ struct TcConfig {
   size_t smem, ws_counters_off, ws_partials_off, ws_bytes;
 };
 cudaError_t tc_configure(TcConfig& c, int num_sms);
-// Encode the TMA descriptors (CUtensorMap, 128 bytes each) for one weight set.
-bool tc_encode_maps(const TcConfig& c, const uint8_t* wp, const uint8_t* ws, void* map_w,
-                    void* map_s);
+// Encode the TMA descriptors (CUtensorMap, 128 bytes each) of one weight set:
+// codes in boxes of 128 bytes x box_rows rows (128-byte swizzle), scales in
+// boxes of 16 bytes x box_rows rows.
+bool encode_weight_maps(int N, int K, int box_rows, const uint8_t* wp, const uint8_t* ws,
+                        void* map_w, void* map_s);
+bool tensor_maps_supported();
 cudaError_t launch_tc(const TcConfig& c, const void* map_w, const void* map_s, const float* gs,
                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
                       bool stall, cudaStream_t st);
+
+// Register-direct warp-MMA variant (k_mma.cu).
+struct MmaConfig {
+  int M, N, K;
+  int tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, grid;
+  bool split;
+  size_t smem, ws_counters_off, ws_partials_off, ws_bytes;
+};
+cudaError_t mma_configure(MmaConfig& c, int num_sms);
+cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s, const float* gs,
+                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
+                       bool stall, cudaStream_t st);
+constexpr int kMmaTileRows = 256;
 
 }  // namespace nvfp4

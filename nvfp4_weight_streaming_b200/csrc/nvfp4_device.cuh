@@ -82,4 +82,77 @@ __device__ __forceinline__ uint32_t ld_stream_u16(const void* p) {
   return r;
 }
 
+// ---- shared memory barriers and TMA ----------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(b), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(b) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes)
+               : "memory");
+}
+// Non-blocking-forever probe of an mbarrier phase (the hardware may suspend
+// the thread for a bounded time inside try_wait).
+__device__ __forceinline__ bool mbar_test(uint32_t b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(b), "r"(parity) : "memory");
+  return ok != 0;
+}
+// 2D tiled TMA load into shared memory, completing on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// bar.red.and over `count` threads: every participant gets the AND of `ok`.
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.b32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r) : "r"(ok ? 1u : 0u), "r"(id), "r"(count) : "memory");
+  return r != 0;
+}
+// ---- X as f16 planes ------------------------------------------------------------
+// Exponent of a nonzero finite bf16 value and its 8-bit significand (128..255).
+__device__ __forceinline__ int bf16_exp(uint32_t b, uint32_t& sig) {
+  const uint32_t e8 = (b >> 7) & 0xFFu, mant = b & 0x7Fu;
+  if (e8) { sig = 0x80u | mant; return int(e8) - 127; }
+  const int msb = 31 - __clz(int(mant));
+  sig = mant << (7 - msb);
+  return msb - 133;
+}
+// f16 bits of sign * sig/128 * 2^t for a normal f16 exponent t (else 0).
+__device__ __forceinline__ uint32_t make_f16(uint32_t sign, int t, uint32_t sig) {
+  if (t < -14 || t > 15) return 0;
+  return (sign << 15) | (uint32_t(t + 15) << 10) | ((sig & 0x7Fu) << 3);
+}
+
+// Number of work-range boundaries floor(c * L / W), c in [1, W), lying in (lo, hi].
+__device__ __forceinline__ long long boundaries_in(long long lo, long long hi, long long L, long long W) {
+  if (hi <= lo) return 0;
+  long long cmin = ((lo + 1) * W + L - 1) / L;
+  long long cmax = ((hi + 1) * W + L - 1) / L - 1;
+  if (cmin < 1) cmin = 1;
+  if (cmax > W - 1) cmax = W - 1;
+  return cmax >= cmin ? cmax - cmin + 1 : 0;
+}
+
 }  // namespace nvfp4

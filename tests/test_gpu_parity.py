@@ -268,14 +268,15 @@ def test_linear_k_zero_writes_zeros_and_n_zero_is_noop():
     nv.nvfp4_linear_destroy(plan)
 
 
-def test_tc_forced_timeout_reports_status_and_recovers():
+@pytest.mark.parametrize("variant", [nv.NVFP4_VARIANT_TC, nv.NVFP4_VARIANT_MMA])
+def test_forced_timeout_reports_status_and_recovers(variant):
     """Test-only flag: the TMA producer never signals, every bounded wait runs
     out, the kernel reports NVFP4_ERR_TIMEOUT through the status word and
     returns; the same workspace then serves a normal run."""
     w = tiny_weights()
     X = synth.x_bf16(synth.WORKLOADS["tiny"], 1)
     dev_id = torch.cuda.current_device()
-    plan = nv.nvfp4_linear_plan(1, w.N, w.K, dev_id, nv.NVFP4_VARIANT_TC | nv.NVFP4_PLAN_TEST_STALL)
+    plan = nv.nvfp4_linear_plan(1, w.N, w.K, dev_id, variant | nv.NVFP4_PLAN_TEST_STALL)
     try:
         wsb = nv.nvfp4_linear_workspace_bytes(plan)
         ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
@@ -287,7 +288,7 @@ def test_tc_forced_timeout_reports_status_and_recovers():
     finally:
         nv.nvfp4_linear_destroy(plan)
     y_ref, ad = oracle.linear(w.packed_h, w.scales_h, w.gs, X, 1, w.N, w.K)
-    got, ok, _ = run_linear(w, X, nv.NVFP4_VARIANT_TC)
+    got, ok, _ = run_linear(w, X, variant)
     assert ok
     check_tolerance(got, y_ref, ad)
 
