@@ -118,6 +118,40 @@ nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
                               const void* x, void* y, void* workspace,
                               size_t ws_bytes, void* stream);
 
+/* Size of the fixed device scratch area behind nvfp4_linear_run_static. */
+#define NVFP4_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* nvfp4_linear_run without a caller workspace and without allocating. The
+ * pages define only the linear itself (as for nvfp4_linear_run); this entry
+ * point has no counterpart there. It serves callers that cannot allocate
+ * device memory at the point of the call: an engine that reserved nearly
+ * all of HBM up front (weights, KV cache) and forbids allocation while
+ * serving, a plain C host with no device allocator of its own, or a latency
+ * path where cudaMalloc/cudaFree would stall (cudaFree synchronises the
+ * device). The split-K scratch (status word, per-tile counters, partial
+ * sums) lives instead in one fixed array of NVFP4_STATIC_SCRATCH_BYTES
+ * inside the library, one per device.
+ *   - Same arguments, layout and errors as nvfp4_linear_run, minus the
+ *     workspace. Returns WORKSPACE, launching nothing, if the plan needs more
+ *     than NVFP4_STATIC_SCRATCH_BYTES (nvfp4_linear_workspace_bytes).
+ *   - status_out: optional device pointer (uint32, 4-byte aligned). After
+ *     the kernel, the run's status word is copied there on `stream`: 0 if
+ *     every device wait completed, nonzero if one timed out (then Y is
+ *     unspecified). NULL skips the copy.
+ *   - The first call on a device looks up the array's address with that
+ *     device current, which may load the library's device code there; make
+ *     that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves the last call's
+ *     contents in it; each call clears, on `stream`, the part that must start
+ *     at zero (status word and counters). Calls on one stream are therefore
+ *     ordered and safe; two calls that overlap in time on one device (other
+ *     streams, other host threads) race on the array and give wrong results.
+ *   - Allocates no memory: no cudaMalloc/cudaFree, no library allocator. */
+nvfp4_status nvfp4_linear_run_static(nvfp4_plan_t plan, const uint8_t* w_packed,
+                                     const uint8_t* w_scales, const float* w_global,
+                                     const void* x, void* y, unsigned* status_out,
+                                     void* stream);
+
 /* Synchronise `stream`, then report: CUDA if the stream holds an error,
  * TIMEOUT if a kernel of this plan recorded a device-wait timeout in the
  * workspace status word (the word is cleared), else OK. workspace may be NULL

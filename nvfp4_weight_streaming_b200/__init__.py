@@ -23,7 +23,8 @@ __all__ = [
     "NVFP4_PLAN_SPLITK_SHIFT", "NVFP4_PLAN_TEST_STALL",
     "Nvfp4Error", "lib", "library_path",
     "nvfp4_linear_plan", "nvfp4_linear_workspace_bytes", "nvfp4_linear_variant",
-    "nvfp4_linear_split_k", "nvfp4_linear_run", "nvfp4_linear_status", "nvfp4_linear_destroy",
+    "nvfp4_linear_split_k", "nvfp4_linear_run", "nvfp4_linear_run_static",
+    "NVFP4_STATIC_SCRATCH_BYTES", "nvfp4_linear_status", "nvfp4_linear_destroy",
     "nvfp4_pack_check", "nvfp4_quantize", "nvfp4_status_string", "EXPORTS",
 ]
 
@@ -42,6 +43,7 @@ NVFP4_VARIANT_MMA = 2
 NVFP4_VARIANT_TC = 3
 NVFP4_PLAN_SPLITK_SHIFT = 8
 NVFP4_PLAN_TEST_STALL = 0x40000000
+NVFP4_STATIC_SCRATCH_BYTES = 16 << 20
 
 _c = ctypes
 _P = _c.c_void_p
@@ -53,6 +55,7 @@ EXPORTS = {
     "nvfp4_linear_variant": (_c.c_int, [_P]),
     "nvfp4_linear_split_k": (_c.c_int, [_P]),
     "nvfp4_linear_run": (_c.c_int, [_P, _P, _P, _P, _P, _P, _P, _c.c_size_t, _P]),
+    "nvfp4_linear_run_static": (_c.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "nvfp4_linear_status": (_c.c_int, [_P, _P, _P]),
     "nvfp4_linear_destroy": (None, [_P]),
     "nvfp4_pack_check": (_c.c_int, [_P, _P, _P, _c.c_int, _c.c_int, _P, _P, _P]),
@@ -148,6 +151,16 @@ def nvfp4_linear_run(plan, w_packed, w_scales, w_global, x, y, workspace=None, w
     s = lib().nvfp4_linear_run(plan, _ptr(w_packed), _ptr(w_scales), _ptr(w_global), _ptr(x),
                                _ptr(y), _ptr(workspace), ws_bytes, _stream(stream))
     return _check(s, "nvfp4_linear_run") if check else s
+
+
+def nvfp4_linear_run_static(plan, w_packed, w_scales, w_global, x, y, status_out=None,
+                            stream=None, check: bool = True) -> int:
+    """Launch Y = X W^T with the split-K scratch in the library's fixed device
+    array instead of a caller workspace (nothing is allocated). status_out: an
+    optional device uint32 that receives the run's status word."""
+    s = lib().nvfp4_linear_run_static(plan, _ptr(w_packed), _ptr(w_scales), _ptr(w_global),
+                                      _ptr(x), _ptr(y), _ptr(status_out), _stream(stream))
+    return _check(s, "nvfp4_linear_run_static") if check else s
 
 
 def nvfp4_linear_status(plan, workspace=None, stream=None) -> int:

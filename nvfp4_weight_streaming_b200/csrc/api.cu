@@ -13,6 +13,10 @@
 #include <mutex>
 #include <new>
 
+// Fixed split-K scratch behind nvfp4_linear_run_static: one copy per device
+// (module globals are per device), shared by every call on that device.
+static __device__ __align__(256) unsigned char g_static_scratch[NVFP4_STATIC_SCRATCH_BYTES];
+
 namespace {
 // TMA descriptors of one weight set, keyed by its two device pointers.
 struct MapEntry {
@@ -48,9 +52,25 @@ nvfp4_status check_device(int device) {
   return cur == device ? NVFP4_OK : NVFP4_ERR_INVALID_ARG;
 }
 
-// Which variant AUTO takes for a shape: the fastest measured on B200 for
-// that (M, N, K) class among those that can run it.
-// Measured on B200 for the 5120 x 34816 projection: the CUDA-core GEMV is
+// Device address of g_static_scratch on `device`, which must be current. The
+// first call per device looks it up (this may load the module there).
+constexpr int kMaxScratchDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxScratchDevices] = {};
+
+nvfp4_status static_scratch_address(int device, void** out) {
+  if (device < 0 || device >= kMaxScratchDevices) return NVFP4_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> g(g_scratch_mu);
+  if (!g_scratch_addr[device]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_static_scratch) != cudaSuccess || !a) return NVFP4_ERR_CUDA;
+    g_scratch_addr[device] = a;
+  }
+  *out = g_scratch_addr[device];
+  return NVFP4_OK;
+}
+
+// Which variant AUTO takes for a shape, measured on B200 for the 5120 x 34816 projection: the CUDA-core GEMV is
 // fastest at M = 1, the mma.sync pipeline up to M = 8, the tcgen05 pipeline
 // beyond (its MMA cost does not grow with the token count).
 int auto_variant(int M, int N, int K) {
@@ -294,6 +314,39 @@ nvfp4_status nvfp4_quantize(const float* w, int N, int K, uint8_t* w_packed, uin
   cudaError_t e = nvfp4::launch_quantize(w, N, K, w_packed, w_scales, w_global, d_bad, sms,
                                          static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status nvfp4_linear_run_static(nvfp4_plan_t plan, const uint8_t* w_packed,
+                                     const uint8_t* w_scales, const float* w_global,
+                                     const void* x, void* y, unsigned* status_out,
+                                     void* stream) {
+  if (!plan) return NVFP4_ERR_INVALID_ARG;
+  if (plan->ws_bytes > size_t(NVFP4_STATIC_SCRATCH_BYTES)) return NVFP4_ERR_WORKSPACE;
+  if (status_out && !aligned(status_out, 4)) return NVFP4_ERR_MISALIGNED;
+  nvfp4_status s = check_device(plan->device);
+  if (s != NVFP4_OK) return s;
+  void* scratch = nullptr;
+  s = static_scratch_address(plan->device, &scratch);
+  if (s != NVFP4_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Status word and per-tile counters must start at zero; the partial sums
+  // are written before they are read.
+  size_t zeroed = plan->ws_bytes;
+  if (plan->variant == int(NVFP4_VARIANT_MMA) && plan->mma.ws_partials_off < zeroed)
+    zeroed = plan->mma.ws_partials_off;
+  if (plan->variant == int(NVFP4_VARIANT_TC) && plan->tc.ws_partials_off < zeroed)
+    zeroed = plan->tc.ws_partials_off;
+  if (zeroed > 0 && cudaMemsetAsync(scratch, 0, zeroed, st) != cudaSuccess) return NVFP4_ERR_CUDA;
+  s = nvfp4_linear_run(plan, w_packed, w_scales, w_global, x, y, scratch,
+                       size_t(NVFP4_STATIC_SCRATCH_BYTES), stream);
+  if (s != NVFP4_OK) return s;
+  if (status_out) {
+    const cudaError_t e = plan->ws_bytes > 0
+        ? cudaMemcpyAsync(status_out, scratch, sizeof(unsigned), cudaMemcpyDeviceToDevice, st)
+        : cudaMemsetAsync(status_out, 0, sizeof(unsigned), st);
+    if (e != cudaSuccess) return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
 }
 
 }  // extern "C"

@@ -1,0 +1,118 @@
+"""nvfp4_linear_run_static: the linear with its split-K scratch in the
+library's fixed device array, checked against nvfp4_linear_run with a caller
+workspace on the same plan. Two calls in a row must both match (the second
+one finds the first one's leftovers in the shared array).
+
+Collected last on purpose: it must pass in a fresh process and after every
+other test has used the device.
+"""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_weight_streaming_b200 as nv
+import oracle
+import synth
+from tests.gpu_util import Guarded, Weights, check_tolerance, dev, host_u16, run_linear
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # (variant, M, N, K): split-K plans that use the scratch, and one that needs none
+    (nv.NVFP4_VARIANT_MMA, 4, 1024, 8192),
+    (nv.NVFP4_VARIANT_TC, 16, 1024, 8192),
+    (nv.NVFP4_VARIANT_AUTO, 3, 777, 1280),
+    (nv.NVFP4_VARIANT_GEMV, 1, 520, 512),
+]
+
+
+def _problem(M, N, K, seed):
+    W = synth.normal_f32(N * K, 0.02, seed=seed, stream=7).reshape(N, K)
+    packed, scales, gs = oracle.quantize(W)
+    X = synth.x_bf16_custom(synth.X_OUTLIERS, M, K, seed=seed + 1, n_outliers=4, gain=20.0)
+    return Weights(packed, scales, gs), X
+
+
+@pytest.mark.parametrize("variant,M,N,K", CASES)
+def test_static_scratch_matches_workspace_entry(variant, M, N, K):
+    w, X = _problem(M, N, K, seed=11 + M)
+    _, ad = oracle.linear(w.packed_h, w.scales_h, w.gs, X, M, N, K)
+    plan = nv.nvfp4_linear_plan(M, N, K, torch.cuda.current_device(), variant)
+    try:
+        wsb = nv.nvfp4_linear_workspace_bytes(plan)
+        assert wsb <= nv.NVFP4_STATIC_SCRATCH_BYTES
+        if variant in (nv.NVFP4_VARIANT_MMA, nv.NVFP4_VARIANT_TC):
+            assert nv.nvfp4_linear_split_k(plan) > 1 and wsb > 256, "case must use split-K scratch"
+        y_ws, ok, _ = run_linear(w, X, plan=plan)
+        assert ok
+        y_ref = oracle.bf16_bits_to_f64(y_ws)
+
+        xd = dev(X)
+        stream = torch.cuda.current_stream()
+        status = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+        outs = []
+        for call in range(2):
+            y = Guarded(M * N)
+            nv.nvfp4_linear_run_static(plan, w.packed, w.scales, w.gsd, xd, y.view,
+                                       status[call:call + 1], stream)
+            outs.append(y)
+        torch.cuda.synchronize()
+        assert status.tolist() == [0, 0], "device wait status %s" % status.tolist()
+        for y in outs:
+            assert y.guards_intact()
+            check_tolerance(host_u16(y.view).reshape(M, N), y_ref, ad)
+    finally:
+        nv.nvfp4_linear_destroy(plan)
+
+
+def test_static_scratch_rejects_plans_beyond_its_size():
+    """A plan whose workspace exceeds the fixed array is refused with
+    WORKSPACE and launches nothing."""
+    dev_id = torch.cuda.current_device()
+    found = None
+    sizes = []
+    for v in (nv.NVFP4_VARIANT_TC, nv.NVFP4_VARIANT_MMA):
+        for N, K in ((1024, 65536), (2048, 65536), (4096, 65536), (8192, 65536),
+                     (16384, 32768), (32768, 16384)):
+            try:
+                p = nv.nvfp4_linear_plan(16, N, K, dev_id, v)
+            except nv.Nvfp4Error:
+                continue
+            wsb = nv.nvfp4_linear_workspace_bytes(p)
+            sizes.append((v, N, K, wsb))
+            if wsb > nv.NVFP4_STATIC_SCRATCH_BYTES and found is None:
+                found = (p, N, K)
+            else:
+                nv.nvfp4_linear_destroy(p)
+    assert found is not None, "no candidate plan exceeds the array: %s" % sizes
+    p, N, K = found
+    try:
+        d = torch.empty(16, dtype=torch.uint8, device="cuda")
+        y = Guarded(16 * N)
+        s = nv.nvfp4_linear_run_static(p, d, d, d, d, y.view, None, None, check=False)
+        assert s == nv.NVFP4_ERR_WORKSPACE
+        torch.cuda.synchronize()
+        assert y.guards_intact() and bool((y.view == 0x5A5A).all())
+    finally:
+        nv.nvfp4_linear_destroy(p)
+
+
+def test_static_scratch_argument_errors():
+    L = nv.lib()
+    assert L.nvfp4_linear_run_static(None, None, None, None, None, None, None, None) == \
+        nv.NVFP4_ERR_INVALID_ARG
+    M, N, K = 4, 1024, 8192
+    w, X = _problem(M, N, K, seed=5)
+    plan = nv.nvfp4_linear_plan(M, N, K, torch.cuda.current_device(), nv.NVFP4_VARIANT_MMA)
+    try:
+        y = Guarded(M * N)
+        st = torch.zeros(2, dtype=torch.int32, device="cuda")
+        odd = st.data_ptr() + 1
+        s = nv.nvfp4_linear_run_static(plan, w.packed, w.scales, w.gsd, dev(X), y.view, odd,
+                                       None, check=False)
+        assert s == nv.NVFP4_ERR_MISALIGNED
+        s = nv.nvfp4_linear_run_static(plan, w.packed, w.scales, w.gsd, None, y.view, None,
+                                       None, check=False)
+        assert s == nv.NVFP4_ERR_INVALID_ARG
+    finally:
+        nv.nvfp4_linear_destroy(plan)
