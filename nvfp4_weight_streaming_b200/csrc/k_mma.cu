@@ -62,12 +62,19 @@ constexpr int NCW = 16;                    // consumer warps (16 rows each)
 constexpr int WARP_SETTLE = NCW + 1;       // warp 0 producer, 1..16 consumers, 17 settler
 constexpr int NUM_THREADS = (NCW + 2) * 32;
 constexpr int QN = 8;                      // split-tile queue slots (consumers -> settler)
-constexpr int MAX_PIECES = 62;             // pieces of one tile the settler can list
-constexpr int NSTAGE = 4;
+constexpr int MAX_PIECES = 62;             // pieces of one tile that can be listed
+constexpr int FAST_MAX = 3;                // other pieces the in-loop finish can add
+constexpr int LIST_MAX = 32;               // row groups whose sum waits for the end phase
+constexpr int NSTAGE_MIN = 4;             // ring depth the X budget is planned with
+constexpr int NSTAGE_MAX = 8;             // deeper rings use what X leaves free
 constexpr int W_BYTES = TROWS * KS / 2;    // 32768
 constexpr int S_BYTES = TROWS * KS / 16;   // 4096
-constexpr int RING_BYTES = NSTAGE * (W_BYTES + S_BYTES);
-constexpr int MISC_BYTES = 640;
+constexpr int STAGE_BYTES = W_BYTES + S_BYTES;
+constexpr int MISC_BYTES = 1024;
+// misc area: barriers [0,256) (full, empty, qfull, qempty: 8 each), emax [256,320),
+// flags [320,336) (need_lo, abort, list count), skip masks [336,368),
+// piece slots [384,640), end-phase list [640,896)
+constexpr int MISC_EMAX = 256, MISC_FLAGS = 320, MISC_SKIP = 336, MISC_PIECES = 384, MISC_LIST = 640;
 constexpr int BAR_XISSUED = 2;             // producer waits until X loads are issued
 constexpr int MAXC = 6;                    // X chunks (8 elements) per consumer thread
 constexpr int LO_SHIFT = 29;
@@ -77,7 +84,7 @@ constexpr uint32_t ST_TIMEOUT_PRODUCER = 1u, ST_TIMEOUT_CONSUMER = 2u, ST_TIMEOU
                    ST_TIMEOUT_DRAIN = 16u;
 
 struct Params {
-  int M, N, K, tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax;
+  int M, N, K, tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, nstage;
   const float* gs;
   const uint16_t* x;
   uint16_t* y;
@@ -88,11 +95,13 @@ struct Params {
   int stall;
 };
 
-// Byte offset of X element k (local to the slice) inside a column: 8-byte
-// granules q = k/4 are XOR-swizzled by bits 4..5 of q.
+// Byte offset of X element k (local to the slice) inside a column: groups of
+// 64 elements take 136 bytes (8 bytes of padding), so the four lanes t of an
+// MMA, which read groups 4s+t of step s, start on different banks and the
+// offsets of the sixteen MMAs of a step are immediates.
+constexpr int XGROUP_BYTES = 136;
 __device__ __forceinline__ uint32_t x_off(int k) {
-  const int q = k >> 2;
-  return uint32_t(((q ^ ((q >> 4) & 3)) << 3) | ((k & 3) << 1));
+  return uint32_t(XGROUP_BYTES * (k >> 6) + 2 * (k & 63));
 }
 
 __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -119,6 +128,53 @@ __device__ __forceinline__ bool wait_bar(uint32_t b, uint32_t parity, volatile i
   }
 }
 
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* a) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+// Slots of the pieces of `tile` in k order (slice, then ordinal); returns
+// their number (at most MAX_PIECES are listed).
+__device__ __forceinline__ int list_pieces(const Params& p, int tile, uint32_t* out) {
+  int n = 0;
+  for (int s2 = 0; s2 < p.S; ++s2) {
+    const int cnt2 = p.ks_base + (s2 < p.ks_rem ? 1 : 0);
+    const long long L2 = (long long)p.tiles * cnt2;
+    const int np = 1 + int(boundaries_in((long long)tile * cnt2, (long long)(tile + 1) * cnt2 - 1, L2, p.P));
+    for (int o = 0; o < np && n < MAX_PIECES; ++o)
+      out[n++] = uint32_t(((long long)tile * p.S + s2) * p.pmax + o);
+  }
+  return n;
+}
+
+// Y rows of the row groups in `gmask` of `tile` = sum of all pieces in k
+// order (first piece first), for threads tid, tid + nth, ...
+__device__ __forceinline__ void sum_pieces(const Params& p, int tile, uint32_t gmask,
+                                           const uint32_t* pieces, int np, int tid, int nth) {
+  const float gs = *p.gs;
+  const int MT = p.M * TROWS;
+  const int nval = __popc(gmask) * 16 * p.M;
+  for (int u = tid; u < nval; u += nth) {
+    const int rr = u & 15, rest = u >> 4;
+    const int m = rest % p.M, gi = rest / p.M;
+    const int grp = __fns(gmask, 0, gi + 1);
+    const int row = grp * 16 + rr;
+    const float* base = p.partials + size_t(m) * TROWS + row;
+    float sum = __ldcg(base + size_t(pieces[0]) * MT);
+    int o = 1;
+    for (; o + 3 < np; o += 4) {
+      const float v1 = __ldcg(base + size_t(pieces[o]) * MT), v2 = __ldcg(base + size_t(pieces[o + 1]) * MT);
+      const float v3 = __ldcg(base + size_t(pieces[o + 2]) * MT), v4 = __ldcg(base + size_t(pieces[o + 3]) * MT);
+      sum += v1; sum += v2; sum += v3; sum += v4;
+    }
+    for (; o < np; ++o) sum += __ldcg(base + size_t(pieces[o]) * MT);
+    const int n = tile * TROWS + row;
+    if (n < p.N) p.y[size_t(m) * p.N + n] = float_to_bf16_bits(gs * sum);
+  }
+}
+
 __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Params& p) {
   const long long t0 = clock64();
   while (!mbar_test(b, parity)) {
@@ -135,7 +191,8 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
 // instead of sixteen MMAs serialised on one accumulator.
 template <int NTILE>
 __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* ss, int r, float (*acc)[4],
-                                             const uint8_t* xcol, uint32_t xstride, int kloc, int t) {
+                                             const uint8_t* sx, const uint32_t* xcol, const bool* xon,
+                                             int kloc, int t) {
   const int r1 = r + 8;
   // chunks 2t, 2t+1 of each row; the TMA 128-byte swizzle puts chunk c of row
   // r at position c ^ (r & 7)
@@ -147,11 +204,15 @@ __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* s
   const uint32_t s1 = *reinterpret_cast<const uint32_t*>(ss + r1 * 16 + 4 * t);
   const uint32_t w0[8] = {c00.x, c00.y, c00.z, c00.w, c01.x, c01.y, c01.z, c01.w};
   const uint32_t w1[8] = {c10.x, c10.y, c10.z, c10.w, c11.x, c11.y, c11.z, c11.w};
-  const uint32_t s0lo = e4m3x2_to_f16x2(s0), s0hi = e4m3x2_to_f16x2(s0 >> 16);
-  const uint32_t s1lo = e4m3x2_to_f16x2(s1), s1hi = e4m3x2_to_f16x2(s1 >> 16);
-  const uint32_t sc0[4] = {bcast_lo(s0lo), bcast_hi(s0lo), bcast_lo(s0hi), bcast_hi(s0hi)};
-  const uint32_t sc1[4] = {bcast_lo(s1lo), bcast_hi(s1lo), bcast_lo(s1hi), bcast_hi(s1hi)};
-  const int qbase = (kloc >> 2) + 16 * t;
+  // each scale byte duplicated, then converted: f16x2 {s, s}
+  const uint32_t d0a = __byte_perm(s0, 0, 0x1100), d0b = __byte_perm(s0, 0, 0x3322);
+  const uint32_t d1a = __byte_perm(s1, 0, 0x1100), d1b = __byte_perm(s1, 0, 0x3322);
+  const uint32_t sc0[4] = {e4m3x2_to_f16x2(d0a), e4m3x2_to_f16x2(d0a >> 16), e4m3x2_to_f16x2(d0b),
+                           e4m3x2_to_f16x2(d0b >> 16)};
+  const uint32_t sc1[4] = {e4m3x2_to_f16x2(d1a), e4m3x2_to_f16x2(d1a >> 16), e4m3x2_to_f16x2(d1b),
+                           e4m3x2_to_f16x2(d1b >> 16)};
+  // lane t reads group 4 * (kloc / 256) + t of each X column
+  const uint32_t xg = uint32_t(XGROUP_BYTES * ((kloc >> 6) + t));
 #pragma unroll
   for (int wd = 0; wd < 8; ++wd) {
     uint32_t h0[4], h1[4];
@@ -165,11 +226,11 @@ __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* s
       const uint32_t a1 = hmul2(h1[2 * hh], cc1);      // row g+8, k = 4i, 4i+1
       const uint32_t a2 = hmul2(h0[2 * hh + 1], cc0);  // row g,   k = 4i+2, 4i+3
       const uint32_t a3 = hmul2(h1[2 * hh + 1], cc1);  // row g+8, k = 4i+2, 4i+3
-      const uint32_t off = uint32_t(((qbase + i) ^ t) << 3);
       constexpr int NSET = 4 / NTILE;
 #pragma unroll
       for (int nt = 0; nt < NTILE; ++nt) {
-        const uint2 bb = *reinterpret_cast<const uint2*>(xcol + nt * 8 * xstride + off);
+        uint2 bb = make_uint2(0u, 0u);
+        if (xon[nt]) bb = *reinterpret_cast<const uint2*>(sx + (xcol[nt] + xg) + 8 * i);
         mma16816(acc[(i % NSET) * NTILE + nt], a0, a1, a2, a3, bb.x, bb.y);
       }
     }
@@ -185,8 +246,8 @@ template <int MC, int NTILE>
 __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* sS, const uint8_t* sX,
                                         const int* emax, uint32_t b_full, uint32_t b_empty,
                                         uint32_t b_qfull, uint32_t b_qempty,
-                                        volatile int* abort_flag, int s, int cnt, long long a,
-                                        long long b, long long L, int cw, int lane) {
+                                        volatile int* abort_flag, uint32_t* skip, int s, int cnt,
+                                        int a, int b, int L, int cw, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int r = 16 * cw + g;                           // row of the tile (and r + 8)
   int tok[4];
@@ -209,22 +270,39 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     }
   }
   const float gs = *p.gs;
-  const uint8_t* xcol = sX + size_t(g) * p.xstride;
+  // X column of each token tile for this lane (B column g); shared memory
+  // holds only the 2M used columns: hi plane tokens 0..M-1, then lo plane
+  uint32_t xcol[NTILE];
+  bool xon[NTILE];
+#pragma unroll
+  for (int nt = 0; nt < NTILE; ++nt) {
+    int plane, tk;
+    if (MC == 1) { plane = g >> 2; tk = g & 3; }
+    else if (MC == 2) { plane = nt; tk = g; }
+    else if (NTILE == 4) { plane = nt >> 1; tk = 8 * (nt & 1) + g; }
+    else { plane = 0; tk = 8 * nt + g; }
+    xon[nt] = tk < p.M;
+    xcol[nt] = uint32_t(plane * p.M + (xon[nt] ? tk : 0)) * uint32_t(p.xstride);
+  }
   float acc[4][4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.0f;
-  long long i = 0;                                     // stage counter
-  long long seg_start = a;
+  int st = 0;                                          // ring stage and its phase
+  uint32_t ph = 0;
+  int seg_start = a;
   int nsplit = 0;                                      // split segments handed to the settler
-  for (long long idx = a; idx < b; ++idx, ++i) {
-    const int st = int(i % NSTAGE);
-    const bool ok = wait_bar(b_full + 8 * st, uint32_t(i / NSTAGE) & 1u, abort_flag, p, ST_TIMEOUT_CONSUMER);
+  int tile = a / cnt, j = a - tile * cnt;
+  for (int idx = a; idx < b; ++idx) {
+    const bool ok = wait_bar(b_full + 8 * st, ph, abort_flag, p, ST_TIMEOUT_CONSUMER);
     if (!__all_sync(0xffffffffu, ok)) break;
-    const int tile = int(idx / cnt), j = int(idx % cnt);
-    compute_step<NTILE>(sW + st * W_BYTES, sS + st * S_BYTES, r, acc, xcol, p.xstride, j * KS, t);
+    compute_step<NTILE>(sW + st * W_BYTES, sS + st * S_BYTES, r, acc, sX, xcol, xon, j * KS, t);
     __syncwarp();
     if (lane == 0) mbar_arrive(b_empty + 8 * st);
-    const bool seg_last = (idx + 1 == b) || (j + 1 == cnt);
+    if (++st == p.nstage) { st = 0; ph ^= 1u; }
+    const int jcur = j;
+    const int tcur = tile;
+    if (++j == cnt) { j = 0; ++tile; }
+    const bool seg_last = (idx + 1 == b) || (jcur + 1 == cnt);
     if (!seg_last) continue;
 
     // ------------------------------------------------------ segment epilogue
@@ -273,10 +351,10 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
         v[2 + e][1] = at[1 % NTILE][2 + e] * fh[2 + e] + l3 * fl[2 + e];
       }
     }
-    const long long this_start = seg_start;
+    const int this_start = seg_start;
     seg_start = idx + 1;
-    const bool whole = (p.S == 1) && (this_start == (long long)tile * cnt) && (j + 1 == cnt);
-    const int row0 = tile * TROWS + r, row1 = row0 + 8;
+    const bool whole = (p.S == 1) && (this_start == tcur * cnt) && (jcur + 1 == cnt);
+    const int row0 = tcur * TROWS + r, row1 = row0 + 8;
     if (whole) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -288,85 +366,140 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
       }
       continue;
     }
-    // piece of a split tile: write the partial, then queue it for the settler
+    // piece of a split tile
     const int qs = nsplit % QN;
     if (nsplit >= QN) {
       const bool okq = wait_bar(b_qempty + 8 * qs, uint32_t((nsplit / QN) - 1) & 1u, abort_flag, p,
                                 ST_TIMEOUT_CONSUMER);
       if (!__all_sync(0xffffffffu, okq)) break;
     }
-    const int ord = int(boundaries_in((long long)tile * cnt, this_start, L, p.P));
-    const long long slot = ((long long)tile * p.S + s) * p.pmax + ord;
-    float* part = p.partials + slot * p.M * TROWS;
+    const int ord = int(boundaries_in((long long)tcur * cnt, this_start, L, p.P));
+    bool done_here = false;
+    if (p.S == 1 && ord == 0 && idx + 1 == b) {
+      // The CTA's last segment holds the tile's first k-range. The other
+      // pieces were the first segments of the next CTAs and are usually
+      // counted by now: then this warp adds them to its registers and stores
+      // its rows without writing a partial.
+      const int np = 1 + int(boundaries_in((long long)tcur * cnt, (long long)(tcur + 1) * cnt - 1, L, p.P));
+      if (np - 1 <= FAST_MAX) {
+        uint32_t* ctr = p.counters + tcur * NCW + cw;
+        const uint32_t seen = ld_relaxed_gpu(ctr);
+        if (__all_sync(0xffffffffu, seen == uint32_t(np - 1))) {
+          fence_acq_rel_gpu();                       // with the relaxed load: acquire
+          float sum[4][2];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int m = tok[e];
-      if (m >= 0 && m < p.M) {
-        part[m * TROWS + r] = v[e][0];
-        part[m * TROWS + r + 8] = v[e][1];
+          for (int e = 0; e < 4; ++e) { sum[e][0] = v[e][0]; sum[e][1] = v[e][1]; }
+#pragma unroll
+          for (int o = 1; o <= FAST_MAX; ++o) {
+            if (o < np) {
+              const float* part = p.partials + ((long long)tcur * p.pmax + o) * p.M * TROWS;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int m = tok[e];
+                if (m >= 0 && m < p.M) {
+                  sum[e][0] += __ldcg(part + m * TROWS + r);
+                  sum[e][1] += __ldcg(part + m * TROWS + r + 8);
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int m = tok[e];
+            if (m >= 0 && m < p.M) {
+              if (row0 < p.N) p.y[size_t(m) * p.N + row0] = float_to_bf16_bits(gs * sum[e][0]);
+              if (row1 < p.N) p.y[size_t(m) * p.N + row1] = float_to_bf16_bits(gs * sum[e][1]);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) *reinterpret_cast<volatile uint32_t*>(ctr) = 0u;
+          done_here = true;
+        }
+      }
+    }
+    if (!done_here) {
+      const long long slot = ((long long)tcur * p.S + s) * p.pmax + ord;
+      float* part = p.partials + slot * p.M * TROWS;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int m = tok[e];
+        if (m >= 0 && m < p.M) {
+          part[m * TROWS + r] = v[e][0];
+          part[m * TROWS + r + 8] = v[e][1];
+        }
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(b_qfull + 8 * qs);
+    if (lane == 0) {
+      if (done_here) atomicOr(&skip[qs], 1u << cw);
+      mbar_arrive(b_qfull + 8 * qs);
+    }
     ++nsplit;
   }
 }
 
-// Settler warp: walks the same segments as the consumers; for each split
-// tile, once all consumer warps have written its piece, it bumps the tile's
-// counter; if this CTA brought the last piece it adds all pieces in k order
-// (slice, then ordinal) and stores Y, and resets the counter.
+// Settler warp: walks the same segments as the consumers. For each split
+// piece, once all consumer warps have written their rows (or finished them
+// in place, see the skip mask), it counts the piece on each row group's
+// counter (a gpu-scope fence first: the mbarrier wait ordered the consumers'
+// partial stores before it, and fences are cumulative). Row groups for which
+// this CTA brought the last piece are listed for the end phase, where all
+// warps of the CTA add the pieces; if the list is full the settler adds them
+// itself.
 __device__ __forceinline__ void settle(const Params& p, uint32_t b_qfull, uint32_t b_qempty,
-                                       volatile int* abort_flag, int cnt, long long a, long long b,
-                                       int lane, uint32_t* pieces) {
-  const float gs = *p.gs;
+                                       volatile int* abort_flag, uint32_t* skip, uint32_t* list,
+                                       uint32_t* nlist, uint32_t* pieces, int cnt, int a, int b,
+                                       int lane) {
   int nsplit = 0;
-  long long seg_start = a;
-  for (long long idx = a; idx < b; ++idx) {
-    const int tile = int(idx / cnt), j = int(idx % cnt);
-    if (!((idx + 1 == b) || (j + 1 == cnt))) continue;
-    const long long this_start = seg_start;
+  int seg_start = a;
+  int tile = a / cnt, j = a - tile * cnt;
+  for (int idx = a; idx < b; ++idx) {
+    const int tcur = tile, jcur = j;
+    if (++j == cnt) { j = 0; ++tile; }
+    if (!((idx + 1 == b) || (jcur + 1 == cnt))) continue;
+    const int this_start = seg_start;
     seg_start = idx + 1;
-    const bool whole = (p.S == 1) && (this_start == (long long)tile * cnt) && (j + 1 == cnt);
+    const bool whole = (p.S == 1) && (this_start == tcur * cnt) && (jcur + 1 == cnt);
     if (whole) continue;
     const int qs = nsplit % QN;
     const bool ok = wait_bar(b_qfull + 8 * qs, uint32_t(nsplit / QN) & 1u, abort_flag, p, ST_TIMEOUT_SETTLER);
     if (!__all_sync(0xffffffffu, ok)) return;
-    unsigned last = 0;
+    // total pieces of the tile over all slices
+    int npieces = 0;
+    for (int s2 = 0; s2 < p.S; ++s2) {
+      const int cnt2 = p.ks_base + (s2 < p.ks_rem ? 1 : 0);
+      const long long L2 = (long long)p.tiles * cnt2;
+      npieces += 1 + int(boundaries_in((long long)tcur * cnt2, (long long)(tcur + 1) * cnt2 - 1, L2, p.P));
+    }
+    const uint32_t sk = skip[qs];
+    bool last = false;
+    if (lane < NCW && !((sk >> lane) & 1u)) {
+      __threadfence();
+      const uint32_t old = atomicAdd(&p.counters[tcur * NCW + lane], 1u);
+      last = old == uint32_t(npieces - 1);
+      if (last) __threadfence();                 // with the atomic: acquire the other pieces
+    }
+    const uint32_t lastmask = __ballot_sync(0xffffffffu, last);
+    if (lastmask) {
+      if (*nlist < uint32_t(LIST_MAX)) {
+        if (lane == 0) {
+          list[2 * *nlist] = uint32_t(tcur);
+          list[2 * *nlist + 1] = lastmask;
+          *nlist += 1;
+        }
+      } else {
+        if (lane == 0) pieces[MAX_PIECES] = uint32_t(list_pieces(p, tcur, pieces));
+        __syncwarp();
+        __threadfence();
+        sum_pieces(p, tcur, lastmask, pieces, int(pieces[MAX_PIECES]), lane, 32);
+        if ((lastmask >> lane) & 1u) p.counters[tcur * NCW + lane] = 0u;
+      }
+    }
+    __syncwarp();
     if (lane == 0) {
-      // the tile's pieces in k order (slice, then ordinal) as partial slots
-      int npieces = 0;
-      for (int s2 = 0; s2 < p.S; ++s2) {
-        const int cnt2 = p.ks_base + (s2 < p.ks_rem ? 1 : 0);
-        const long long L2 = (long long)p.tiles * cnt2;
-        const int np = 1 + int(boundaries_in((long long)tile * cnt2, (long long)(tile + 1) * cnt2 - 1, L2, p.P));
-        for (int o = 0; o < np && npieces < MAX_PIECES; ++o)
-          pieces[npieces++] = uint32_t(((long long)tile * p.S + s2) * p.pmax + o);
-      }
-      pieces[MAX_PIECES] = uint32_t(npieces);
-      // the mbarrier wait orders the consumers' partial stores before this
-      // gpu-scope fence (fences are cumulative); then the counter
-      __threadfence();
-      const unsigned old = atomicAdd(&p.counters[tile], 1u);
-      __threadfence();
-      last = (old == unsigned(npieces - 1)) ? 1u : 0u;
+      skip[qs] = 0u;
+      mbar_arrive(b_qempty + 8 * qs);
     }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    __syncwarp();
-    if (last) {
-      const int npieces = int(pieces[MAX_PIECES]);
-      const int MT = p.M * TROWS;
-      for (int u = lane; u < MT; u += 32) {
-        float sum = 0.0f;
-        for (int o = 0; o < npieces; ++o) sum += __ldcg(p.partials + size_t(pieces[o]) * MT + u);
-        const int m = u / TROWS, row = tile * TROWS + (u - m * TROWS);
-        if (row < p.N) p.y[size_t(m) * p.N + row] = float_to_bf16_bits(gs * sum);
-      }
-      __syncwarp();
-      if (lane == 0) atomicExch(&p.counters[tile], 0u);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(b_qempty + 8 * qs);
     ++nsplit;
   }
 }
@@ -377,30 +510,34 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sW = smem;                                     // NSTAGE x 32 KB (1024-aligned)
-  uint8_t* sS = smem + NSTAGE * W_BYTES;                  // NSTAGE x 4 KB
-  uint8_t* sX = sS + NSTAGE * S_BYTES;
+  const int nst = p.nstage;
+  uint8_t* sW = smem;                                     // nst x 32 KB (1024-aligned)
+  uint8_t* sS = smem + nst * W_BYTES;                     // nst x 4 KB
+  uint8_t* sX = sS + nst * S_BYTES;
   uint8_t* misc = sX + size_t(p.ncols) * p.xstride;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(misc);     // full[4] empty[4] qfull[8] qempty[8]
-  int* emax = reinterpret_cast<int*>(misc + 256);          // [16]
-  uint32_t* flags = reinterpret_cast<uint32_t*>(misc + 320);  // [0] need_lo [1] abort
+  uint64_t* bars = reinterpret_cast<uint64_t*>(misc);     // full[8] empty[8] qfull[8] qempty[8]
+  int* emax = reinterpret_cast<int*>(misc + MISC_EMAX);   // [16]
+  uint32_t* flags = reinterpret_cast<uint32_t*>(misc + MISC_FLAGS);  // [0] need_lo [1] abort [2] list count
+  uint32_t* skip = reinterpret_cast<uint32_t*>(misc + MISC_SKIP);    // [QN]
+  uint32_t* pieces = reinterpret_cast<uint32_t*>(misc + MISC_PIECES);  // [MAX_PIECES + 1]
+  uint32_t* list = reinterpret_cast<uint32_t*>(misc + MISC_LIST);    // [LIST_MAX][2]
   volatile int* abort_flag = reinterpret_cast<volatile int*>(flags + 1);
-  const uint32_t b_full = smem_u32(bars), b_empty = b_full + 8 * NSTAGE;
-  const uint32_t b_qfull = b_empty + 8 * NSTAGE, b_qempty = b_qfull + 8 * QN;
+  const uint32_t b_full = smem_u32(bars), b_empty = b_full + 8 * NSTAGE_MAX;
+  const uint32_t b_qfull = b_empty + 8 * NSTAGE_MAX, b_qempty = b_qfull + 8 * QN;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int s = blockIdx.x / p.P, c = blockIdx.x % p.P;
   const int cnt = p.ks_base + (s < p.ks_rem ? 1 : 0);
   const int ks0 = s * p.ks_base + min(s, p.ks_rem);
   const int klen = cnt * KS, k0e = ks0 * KS;
-  const int mcols = MC == 1 ? 4 : (MC == 2 ? 8 : 16);    // columns per plane
-  const long long L = (long long)p.tiles * cnt;
-  const long long a = (long long)c * L / p.P, b = (long long)(c + 1) * L / p.P;
+  const int L = p.tiles * cnt;
+  const int a = int((long long)c * L / p.P), b = int((long long)(c + 1) * L / p.P);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NSTAGE; ++i) { mbar_init(b_full + 8 * i, 1); mbar_init(b_empty + 8 * i, NCW); }
+    for (int i = 0; i < nst; ++i) { mbar_init(b_full + 8 * i, 1); mbar_init(b_empty + 8 * i, NCW); }
     for (int i = 0; i < QN; ++i) { mbar_init(b_qfull + 8 * i, NCW); mbar_init(b_qempty + 8 * i, 1); }
     for (int m = 0; m < 16; ++m) emax[m] = INT_MIN;
-    flags[0] = 0u; flags[1] = 0u;
+    flags[0] = 0u; flags[1] = 0u; flags[2] = 0u;
+    for (int i = 0; i < QN; ++i) skip[i] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -412,28 +549,30 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     // they are not queued behind the weight stream
     named_bar(BAR_XISSUED, (NCW + 1) * 32);
     if (lane == 0) {
-      long long n_issued = 0;
+      int n_issued = 0;
       if (!p.stall) {
-        for (long long idx = a; idx < b; ++idx, ++n_issued) {
-          const int tile = int(idx / cnt), j = int(idx % cnt);
-          const int st = int(n_issued % NSTAGE);
-          const uint32_t ph = uint32_t(n_issued / NSTAGE) & 1u;
+        int tile = a / cnt, j = a - tile * cnt, st = 0;
+        uint32_t ph = 0;
+        for (int idx = a; idx < b; ++idx, ++n_issued) {
           if (!wait_bar(b_empty + 8 * st, ph ^ 1u, abort_flag, p, ST_TIMEOUT_PRODUCER)) break;
-          mbar_expect_tx(b_full + 8 * st, W_BYTES + S_BYTES);
+          mbar_expect_tx(b_full + 8 * st, STAGE_BYTES);
           tma_load_2d(smem_u32(sW + st * W_BYTES), &tm_w, (ks0 + j) * (KS / 2), tile * TROWS, b_full + 8 * st);
           tma_load_2d(smem_u32(sS + st * S_BYTES), &tm_s, (ks0 + j) * (KS / 16), tile * TROWS, b_full + 8 * st);
+          if (++j == cnt) { j = 0; ++tile; }
+          if (++st == nst) { st = 0; ph ^= 1u; }
         }
       }
       if (*abort_flag) {
-        const long long first = n_issued > NSTAGE ? n_issued - NSTAGE : 0;
-        for (long long i = first; i < n_issued; ++i)
-          drain_bar(b_full + 8 * int(i % NSTAGE), uint32_t(i / NSTAGE) & 1u, p);
+        // wait (bounded) for the loads still in flight before leaving
+        const int first = n_issued > nst ? n_issued - nst : 0;
+        for (int i = first; i < n_issued; ++i)
+          drain_bar(b_full + 8 * (i % nst), uint32_t(i / nst) & 1u, p);
       }
     }
     __syncwarp();
   } else if (warp == WARP_SETTLE) {
     // ---------------------------------------------------------------- settler
-    settle(p, b_qfull, b_qempty, abort_flag, cnt, a, b, lane, reinterpret_cast<uint32_t*>(misc + 384));
+    settle(p, b_qfull, b_qempty, abort_flag, skip, list, flags + 2, pieces, cnt, a, b, lane);
   } else {
     // ------------------------------------------------ consumers: stage X first
     const int ctid = threadIdx.x - 32;                    // 0 .. NCW*32-1
@@ -488,19 +627,11 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
         lo_used |= (lo[0] | lo[1] | lo[2] | lo[3]) != 0u;
         const uint32_t o0 = x_off(8 * kc), o1 = x_off(8 * kc + 4);
         uint8_t* ch = sX + size_t(m) * p.xstride;
-        uint8_t* cl = sX + size_t(mcols + m) * p.xstride;
+        uint8_t* cl = sX + size_t(p.M + m) * p.xstride;
         *reinterpret_cast<uint2*>(ch + o0) = make_uint2(hi[0], hi[1]);
         *reinterpret_cast<uint2*>(ch + o1) = make_uint2(hi[2], hi[3]);
         *reinterpret_cast<uint2*>(cl + o0) = make_uint2(lo[0], lo[1]);
         *reinterpret_cast<uint2*>(cl + o1) = make_uint2(lo[2], lo[3]);
-      }
-    }
-    {
-      const int npad = mcols - p.M;                       // token columns >= M are zero
-      for (int u = ctid; u < 2 * npad * chunks; u += NCT) {
-        const int pr = u / chunks, kc = u - pr * chunks;
-        const int col = (pr < npad) ? (p.M + pr) : (mcols + p.M + pr - npad);
-        *reinterpret_cast<uint4*>(sX + size_t(col) * p.xstride + 16 * kc) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     if (lo_used) atomicOr(&flags[0], 1u);
@@ -509,17 +640,31 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
 
     const int cw = warp - 1;
     if (MC == 1) {
-      consume<1, 1>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, s, cnt, a, b, L, cw, lane);
+      consume<1, 1>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, s, cnt, a, b, L, cw, lane);
     } else if (MC == 2) {
-      consume<2, 2>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, s, cnt, a, b, L, cw, lane);
+      consume<2, 2>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, s, cnt, a, b, L, cw, lane);
     } else {
       if (need_lo)
-        consume<3, 4>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, s, cnt, a, b, L, cw, lane);
+        consume<3, 4>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, s, cnt, a, b, L, cw, lane);
       else
-        consume<3, 2>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, s, cnt, a, b, L, cw, lane);
+        consume<3, 2>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, s, cnt, a, b, L, cw, lane);
     }
   }
   __syncthreads();
+  // ------------------------------------------------------------- end phase
+  // every warp adds the pieces of the row groups this CTA completed last
+  if (!*abort_flag) {
+    const int nl = int(flags[2]);
+    for (int e = 0; e < nl; ++e) {
+      const int tile = int(list[2 * e]);
+      const uint32_t gmask = list[2 * e + 1];
+      if (threadIdx.x == 0) pieces[MAX_PIECES] = uint32_t(list_pieces(p, tile, pieces));
+      __syncthreads();
+      sum_pieces(p, tile, gmask, pieces, int(pieces[MAX_PIECES]), threadIdx.x, NUM_THREADS);
+      if (threadIdx.x < NCW && ((gmask >> threadIdx.x) & 1u)) p.counters[tile * NCW + threadIdx.x] = 0u;
+      __syncthreads();
+    }
+  }
 }
 
 }  // namespace mm
@@ -531,15 +676,20 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
-  const int mcols = c.M <= 4 ? 4 : (c.M <= 8 ? 8 : 16);
-  c.ncols = 2 * mcols;
+  c.ncols = 2 * c.M;                        // hi and lo plane of each token
   c.tiles = (c.N + TROWS - 1) / TROWS;
   const int ksteps = c.K / KS;
-  const long long x_budget = (long long)optin - 1024 - RING_BYTES - MISC_BYTES;
+  const long long x_budget = (long long)optin - 1024 - (long long)NSTAGE_MIN * STAGE_BYTES - MISC_BYTES;
   // largest slice (in steps) whose two X planes fit next to the ring and whose
   // chunks the consumers hold in registers (M * steps * KS / 8 <= MAXC * consumer threads)
+  // column stride: the padded groups, rounded to 32 mod 128 bytes so that
+  // columns g and g+1 start 8 banks apart
+  auto stride_for = [](int ks) {
+    const int base = XGROUP_BYTES * (ks * KS / 64);
+    return ((base - 32 + 127) / 128) * 128 + 32;
+  };
   auto fits = [&](int ks) {
-    return (long long)c.ncols * (ks * KS * 2 + 32) <= x_budget &&
+    return (long long)c.ncols * stride_for(ks) <= x_budget &&
            (long long)c.M * ks * KS / 8 <= (long long)MAXC * NCW * 32;
   };
   if (!fits(1)) return cudaErrorInvalidConfiguration;
@@ -554,7 +704,7 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   c.S = S; c.P = P; c.ks_base = ks_base; c.ks_rem = ks_rem;
   c.grid = S * P;
   c.xk_max = (ks_base + (ks_rem ? 1 : 0)) * KS;
-  c.xstride = c.xk_max * 2 + 32;
+  c.xstride = stride_for(c.xk_max / KS);
   int pmax = 1;
   bool split = S > 1;
   for (int s = 0; s < S; ++s) {
@@ -570,9 +720,15 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   c.pmax = pmax;
   c.split = split;
   if ((long long)S * pmax > MAX_PIECES) return cudaErrorInvalidConfiguration;
-  c.smem = 1024 + size_t(RING_BYTES) + size_t(c.ncols) * c.xstride + MISC_BYTES;
+  {
+    const long long left = (long long)optin - 1024 - (long long)c.ncols * c.xstride - MISC_BYTES;
+    int nst = int(left / STAGE_BYTES);
+    c.nstage = nst < NSTAGE_MAX ? nst : NSTAGE_MAX;
+  }
+  if (c.nstage < NSTAGE_MIN) return cudaErrorInvalidConfiguration;
+  c.smem = 1024 + size_t(c.nstage) * STAGE_BYTES + size_t(c.ncols) * c.xstride + MISC_BYTES;
   c.ws_counters_off = 256;
-  c.ws_partials_off = c.ws_counters_off + ((size_t(c.tiles) * 4 + 255) / 256) * 256;
+  c.ws_partials_off = c.ws_counters_off + ((size_t(c.tiles) * NCW * 4 + 255) / 256) * 256;
   c.ws_bytes = split ? c.ws_partials_off + size_t(c.tiles) * S * pmax * c.M * TROWS * 4 : 256;
   if (c.smem > size_t(optin)) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(k_mma<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
@@ -588,7 +744,7 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
   Params p;
   p.M = c.M; p.N = c.N; p.K = c.K; p.tiles = c.tiles; p.S = c.S; p.P = c.P;
   p.ks_base = c.ks_base; p.ks_rem = c.ks_rem; p.ncols = c.ncols; p.xk_max = c.xk_max;
-  p.xstride = c.xstride; p.pmax = c.pmax;
+  p.xstride = c.xstride; p.pmax = c.pmax; p.nstage = c.nstage;
   p.gs = gs; p.x = x; p.y = y;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   p.status = reinterpret_cast<uint32_t*>(wsb);

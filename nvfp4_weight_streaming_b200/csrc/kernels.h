@@ -51,7 +51,7 @@ cudaError_t launch_tc(const TcConfig& c, const void* map_w, const void* map_s, c
 // Register-direct warp-MMA variant (k_mma.cu).
 struct MmaConfig {
   int M, N, K;
-  int tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, grid;
+  int tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, nstage, grid;
   bool split;
   size_t smem, ws_counters_off, ws_partials_off, ws_bytes;
 };
