@@ -168,7 +168,7 @@ def aggregate(world: int, bytes_per_call: float, sec_per_call_this_rank: float):
 class Problem:
     """One workload on the device: weight copies, X, Y, plan, workspace."""
 
-    def __init__(self, name: str, M: int, variant: int, min_footprint: float):
+    def __init__(self, name: str, M: int, variant: int, min_footprint: float, flags: int = 0):
         import numpy as np
         import torch
         import synth
@@ -196,7 +196,8 @@ class Problem:
         self.x_host = xh
         self.x = torch.from_numpy(xh.view(np.int16)).cuda()
         self.y = torch.empty((M, self.N), dtype=torch.int16, device="cuda")
-        self.plan = nv.nvfp4_linear_plan(M, self.N, self.K, dev, variant)
+        self.plan = nv.nvfp4_linear_plan(M, self.N, self.K, dev, variant | flags)
+        self.flags = flags
         self.variant = nv.nvfp4_linear_variant(self.plan)
         self.split_k = nv.nvfp4_linear_split_k(self.plan)
         self.wsb = nv.nvfp4_linear_workspace_bytes(self.plan)
@@ -356,7 +357,8 @@ def run_ours(args):
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
     peak, peak_kind = peaks()
     variant = {"auto": 0, "gemv": 1, "mma": 2, "tc": 3}[args.variant]
-    pb = Problem(args.workload, args.M, variant, min_footprint=4.2 * l2)
+    flags = 0 if args.no_pdl else nv.NVFP4_PLAN_PDL
+    pb = Problem(args.workload, args.M, variant, min_footprint=4.2 * l2, flags=flags)
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if sampler:
         sampler.start()
@@ -370,7 +372,7 @@ def run_ours(args):
                           [("verify", m) for m in (1, 2, 4, 8, 12, 16)] +
                           [("down", m) for m in (1, 4, 8, 16)] +
                           [("lm_head", m) for m in (1, 8, 16)]):
-            q = Problem(name, M, variant, min_footprint=4.2 * l2)
+            q = Problem(name, M, variant, min_footprint=4.2 * l2, flags=flags)
             s2, _ = time_problem(q, max(args.steps, 200), args.warmup, world)
             g = effective_gbs(q.bytes, s2)
             sweep.append({"workload": name, "M": M, "N": q.N, "K": q.K,
@@ -402,7 +404,10 @@ def run_ours(args):
                        "l2": "inputs larger than L2: %d byte-identical weight copies "
                              "rotated, %.0f MB > %.1f x %.0f MB L2" %
                              (pb.ncopies, pb.footprint / 1e6, pb.footprint / l2, l2 / 1e6),
-                       "launch": "CUDA graphs of back-to-back calls on one stream",
+                       "launch": "CUDA graphs of back-to-back calls on one stream" +
+                                 ("" if args.no_pdl else
+                                  ", programmatic dependent launch (a call streams its weights "
+                                  "while the previous call finishes)"),
                        "parallelism": "replicas x%d" % world},
             "pct_of_measured_peak": 100 * per_gpu / peak,
             "pct_of_nominal_8TBps": 100 * per_gpu / NOMINAL_HBM_GBS,
@@ -472,6 +477,8 @@ def main():
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--variant", choices=["auto", "gemv", "mma", "tc"], default="auto")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-pdl", action="store_true",
+                    help="launch without programmatic dependent launch")
     ap.add_argument("--full-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

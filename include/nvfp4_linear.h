@@ -73,12 +73,16 @@ typedef struct nvfp4_plan_s* nvfp4_plan_t;
  * table of bandwidths measured on B200. */
 #define NVFP4_VARIANT_AUTO 0u
 #define NVFP4_VARIANT_GEMV 1u  /* CUDA-core warp-per-row GEMV, fp32 FMA        */
-#define NVFP4_VARIANT_MMA  2u  /* register-direct warp MMA, split over K       */
+#define NVFP4_VARIANT_MMA  2u  /* TMA ring + warp MMA (m16n8k16), stream-K    */
 #define NVFP4_VARIANT_TC   3u  /* tcgen05 + TMA ring + TMEM accumulators       */
 #define NVFP4_PLAN_VARIANT_MASK 0xFu
-/* Bits 8..15: split-K factor override (0 = let the plan choose). */
-#define NVFP4_PLAN_SPLITK_SHIFT 8u
-#define NVFP4_PLAN_SPLITK_MASK 0xFF00u
+/* Programmatic dependent launch (MMA variant; ignored by the others). The
+ * launch may start while the previous kernel in the stream is still running:
+ * it begins streaming W at once and touches X, Y, w_global and the workspace
+ * only after that kernel has completed. So W (codes and scales) must not be
+ * written by the kernel launched just before it on the same stream. Back to
+ * back calls then overlap one call's tail with the next call's weight stream. */
+#define NVFP4_PLAN_PDL 0x10000u
 /* Test only: the variant's producer never signals, so every bounded device
  * wait runs out and the kernel reports NVFP4_ERR_TIMEOUT through the status
  * word instead of computing. Has no effect on variants without device waits. */

@@ -75,7 +75,6 @@ constexpr int MISC_BYTES = 1024;
 // flags [320,336) (need_lo, abort, list count), skip masks [336,368),
 // piece slots [384,640), end-phase list [640,896)
 constexpr int MISC_EMAX = 256, MISC_FLAGS = 320, MISC_SKIP = 336, MISC_PIECES = 384, MISC_LIST = 640;
-constexpr int BAR_XISSUED = 2;             // producer waits until X loads are issued
 constexpr int MAXC = 6;                    // X chunks (8 elements) per consumer thread
 constexpr int LO_SHIFT = 29;
 constexpr int BAR_CONSUMERS = 1;           // named barrier of the consumer warps
@@ -532,6 +531,9 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
   const int L = p.tiles * cnt;
   const int a = int((long long)c * L / p.P), b = int((long long)(c + 1) * L / p.P);
 
+  // Dependent launches (PDL) may start now: they only stream weights until
+  // this grid has completed.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int i = 0; i < nst; ++i) { mbar_init(b_full + 8 * i, 1); mbar_init(b_empty + 8 * i, NCW); }
     for (int i = 0; i < QN; ++i) { mbar_init(b_qfull + 8 * i, NCW); mbar_init(b_qempty + 8 * i, 1); }
@@ -545,9 +547,7 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
 
   if (warp == 0) {
     // -------------------------------------------------------------- producer
-    // X is read first: wait until every consumer has issued its X loads, so
-    // they are not queued behind the weight stream
-    named_bar(BAR_XISSUED, (NCW + 1) * 32);
+    // Weights do not depend on the previous grid: stream them at once.
     if (lane == 0) {
       int n_issued = 0;
       if (!p.stall) {
@@ -570,11 +570,15 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
       }
     }
     __syncwarp();
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // before the end phase
   } else if (warp == WARP_SETTLE) {
     // ---------------------------------------------------------------- settler
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // counters of the previous grid
     settle(p, b_qfull, b_qempty, abort_flag, skip, list, flags + 2, pieces, cnt, a, b, lane);
   } else {
     // ------------------------------------------------ consumers: stage X first
+    // X, the global scale, Y and the workspace may belong to the previous grid
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int ctid = threadIdx.x - 32;                    // 0 .. NCW*32-1
     constexpr int NCT = NCW * 32;
     const int chunks = klen / 8;
@@ -588,7 +592,6 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
         xv[cc] = *reinterpret_cast<const uint4*>(p.x + size_t(m) * p.K + k0e + 8 * kc);
       }
     }
-    asm volatile("bar.arrive %0, %1;" ::"r"(BAR_XISSUED), "r"((NCW + 1) * 32) : "memory");
 #pragma unroll
     for (int cc = 0; cc < MAXC; ++cc) {
       const int u = ctid + cc * NCT;
@@ -739,7 +742,7 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
 
 cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s, const float* gs,
                        const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
-                       bool stall, cudaStream_t st) {
+                       bool stall, bool pdl, cudaStream_t st) {
   using namespace mm;
   Params p;
   p.M = c.M; p.N = c.N; p.K = c.K; p.tiles = c.tiles; p.S = c.S; p.P = c.P;
@@ -754,10 +757,19 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
   p.stall = stall ? 1 : 0;
   const CUtensorMap& mw = *static_cast<const CUtensorMap*>(map_w);
   const CUtensorMap& ms = *static_cast<const CUtensorMap*>(map_s);
-  if (c.M <= 4) k_mma<1><<<c.grid, NUM_THREADS, c.smem, st>>>(mw, ms, p);
-  else if (c.M <= 8) k_mma<2><<<c.grid, NUM_THREADS, c.smem, st>>>(mw, ms, p);
-  else k_mma<3><<<c.grid, NUM_THREADS, c.smem, st>>>(mw, ms, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(c.grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = c.smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  if (c.M <= 4) return cudaLaunchKernelEx(&cfg, k_mma<1>, mw, ms, p);
+  if (c.M <= 8) return cudaLaunchKernelEx(&cfg, k_mma<2>, mw, ms, p);
+  return cudaLaunchKernelEx(&cfg, k_mma<3>, mw, ms, p);
 }
 
 }  // namespace nvfp4

@@ -58,7 +58,7 @@ struct MmaConfig {
 cudaError_t mma_configure(MmaConfig& c, int num_sms);
 cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s, const float* gs,
                        const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
-                       bool stall, cudaStream_t st);
+                       bool stall, bool pdl, cudaStream_t st);
 constexpr int kMmaTileRows = 256;
 
 }  // namespace nvfp4

@@ -249,6 +249,43 @@ def test_linear_deterministic_and_rows_independent():
         assert np.array_equal(y1, y2), VNAME[v]
 
 
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_pdl_chained_calls_read_the_previous_output(M):
+    """Programmatic dependent launch: each call's X is the previous call's Y,
+    launched back to back on one stream with one shared workspace. Every
+    output must match the oracle applied to the GPU's own previous output, so
+    a call that read X, or reused the workspace, before the previous call had
+    finished would be caught."""
+    K = N = 2048
+    chain = 6
+    ws_h = []
+    for i in range(chain):
+        W = synth.normal_f32(N * K, 1.0 / np.sqrt(K), seed=40 + i, stream=7).reshape(N, K)
+        ws_h.append(oracle.quantize(W))
+    dev_w = [Weights(*q) for q in ws_h]
+    X0 = synth.x_bf16_custom(synth.X_NORMAL, M, K, seed=9)
+    flags = nv.NVFP4_VARIANT_MMA | nv.NVFP4_PLAN_PDL
+    plan = nv.nvfp4_linear_plan(M, N, K, torch.cuda.current_device(), flags)
+    try:
+        wsb = nv.nvfp4_linear_workspace_bytes(plan)
+        ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device="cuda")
+        bufs = [dev(X0)] + [torch.empty((M, N), dtype=torch.int16, device="cuda") for _ in range(chain)]
+        stream = torch.cuda.current_stream()
+        for rep in range(3):
+            for i in range(chain):
+                nv.nvfp4_linear_run(plan, dev_w[i].packed, dev_w[i].scales, dev_w[i].gsd, bufs[i],
+                                    bufs[i + 1], ws, wsb, stream)
+            assert nv.nvfp4_linear_status(plan, ws, stream) == nv.NVFP4_OK
+            for i in range(chain):
+                xin = host_u16(bufs[i]).reshape(M, K)
+                y_ref, ad = oracle.linear(ws_h[i][0], ws_h[i][1], ws_h[i][2], xin, M, N, K)
+                check_tolerance(host_u16(bufs[i + 1]).reshape(M, N), y_ref, ad)
+            for b in bufs[1:]:
+                b.fill_(0x5A5A)
+    finally:
+        nv.nvfp4_linear_destroy(plan)
+
+
 def test_linear_k_zero_writes_zeros_and_n_zero_is_noop():
     w = Weights(np.zeros((8, 0), np.uint8), np.zeros((8, 0), np.uint8), 1.0)
     w.packed = torch.zeros(16, dtype=torch.uint8, device="cuda")
