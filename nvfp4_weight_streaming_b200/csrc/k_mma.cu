@@ -550,14 +550,17 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     // Weights do not depend on the previous grid: stream them at once.
     if (lane == 0) {
       int n_issued = 0;
+      const uint64_t pol = l2_evict_first_policy();
       if (!p.stall) {
         int tile = a / cnt, j = a - tile * cnt, st = 0;
         uint32_t ph = 0;
         for (int idx = a; idx < b; ++idx, ++n_issued) {
           if (!wait_bar(b_empty + 8 * st, ph ^ 1u, abort_flag, p, ST_TIMEOUT_PRODUCER)) break;
           mbar_expect_tx(b_full + 8 * st, STAGE_BYTES);
-          tma_load_2d(smem_u32(sW + st * W_BYTES), &tm_w, (ks0 + j) * (KS / 2), tile * TROWS, b_full + 8 * st);
-          tma_load_2d(smem_u32(sS + st * S_BYTES), &tm_s, (ks0 + j) * (KS / 16), tile * TROWS, b_full + 8 * st);
+          tma_load_2d_hint(smem_u32(sW + st * W_BYTES), &tm_w, (ks0 + j) * (KS / 2), tile * TROWS,
+                           b_full + 8 * st, pol);
+          tma_load_2d_hint(smem_u32(sS + st * S_BYTES), &tm_s, (ks0 + j) * (KS / 16), tile * TROWS,
+                           b_full + 8 * st, pol);
           if (++j == cnt) { j = 0; ++tile; }
           if (++st == nst) { st = 0; ph ^= 1u; }
         }
