@@ -65,17 +65,17 @@ constexpr int QN = 8;                      // split-tile queue slots (consumers 
 constexpr int MAX_PIECES = 62;             // pieces of one tile that can be listed
 constexpr int FAST_MAX = 3;                // other pieces the in-loop finish can add
 constexpr int LIST_MAX = 32;               // row groups whose sum waits for the end phase
-constexpr int NSTAGE_MIN = 4;             // ring depth the X budget is planned with
+constexpr int NSTAGE_MIN = 3;             // ring depth the X budget is planned with
 constexpr int NSTAGE_MAX = 8;             // deeper rings use what X leaves free
 constexpr int W_BYTES = TROWS * KS / 2;    // 32768
 constexpr int S_BYTES = TROWS * KS / 16;   // 4096
 constexpr int STAGE_BYTES = W_BYTES + S_BYTES;
-constexpr int MISC_BYTES = 1024;
+constexpr int MISC_BYTES = 1024 + 4096;
 // misc area: barriers [0,256) (full, empty, qfull, qempty: 8 each), emax [256,320),
 // flags [320,336) (need_lo, abort, list count), skip masks [336,368),
 // piece slots [384,640), end-phase list [640,896)
-constexpr int MISC_EMAX = 256, MISC_FLAGS = 320, MISC_SKIP = 336, MISC_PIECES = 384, MISC_LIST = 640;
-constexpr int MAXC = 6;                    // X chunks (8 elements) per consumer thread
+constexpr int MISC_EMAX = 256, MISC_FLAGS = 320, MISC_SKIP = 336, MISC_PREFLAG = 368, MISC_PIECES = 384,
+              MISC_LIST = 640, MISC_PREBUF = 1024;   // prefetched piece: [M <= 4][TROWS] floats
 constexpr int LO_SHIFT = 29;
 constexpr int BAR_CONSUMERS = 1;           // named barrier of the consumer warps
 
@@ -112,12 +112,15 @@ __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uin
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Bounded mbarrier wait. Between checks of the abort flag and the clock the
+// thread sleeps in try_wait (up to `hint_ns`) rather than spinning, so
+// waiting warps leave the issue slots to the ones computing.
 __device__ __forceinline__ bool wait_bar(uint32_t b, uint32_t parity, volatile int* abort_flag,
-                                         const Params& p, uint32_t who) {
+                                         const Params& p, uint32_t who, uint32_t hint_ns = 2000) {
   if (mbar_test(b, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_test(b, parity)) return true;
+    if (mbar_wait_hint(b, parity, hint_ns)) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > p.timeout) {
       *abort_flag = 1;
@@ -125,6 +128,34 @@ __device__ __forceinline__ bool wait_bar(uint32_t b, uint32_t parity, volatile i
       return false;
     }
   }
+}
+
+// Number of CTA range boundaries floor(c * L / W), c in [1, W), in (lo, hi];
+// 32-bit (configure() checks that L * W fits).
+__device__ __forceinline__ int bnd_in(int lo, int hi, int L, int W) {
+  if (hi <= lo) return 0;
+  int cmin = int((unsigned(lo + 1) * unsigned(W) + unsigned(L) - 1u) / unsigned(L));
+  int cmax = int((unsigned(hi + 1) * unsigned(W) + unsigned(L) - 1u) / unsigned(L)) - 1;
+  if (cmin < 1) cmin = 1;
+  if (cmax > W - 1) cmax = W - 1;
+  return cmax >= cmin ? cmax - cmin + 1 : 0;
+}
+
+// Tile whose first k-range is this CTA's last segment and whose only other
+// piece is the next CTA's first segment (one slice), else -1: the settler
+// fetches that piece into shared memory while the consumers work, so the
+// tile is finished from registers at the end.
+__device__ __forceinline__ int prefetch_tile(const Params& p, int a, int b, int cnt, int L) {
+  if (p.S != 1 || b <= a || p.M > 4) return -1;
+  const int tf = (b - 1) / cnt;
+  if (tf * cnt < a || b >= (tf + 1) * cnt) return -1;
+  return bnd_in(tf * cnt, (tf + 1) * cnt - 1, L, p.P) == 1 ? tf : -1;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* a) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* a) {
@@ -140,8 +171,8 @@ __device__ __forceinline__ int list_pieces(const Params& p, int tile, uint32_t* 
   int n = 0;
   for (int s2 = 0; s2 < p.S; ++s2) {
     const int cnt2 = p.ks_base + (s2 < p.ks_rem ? 1 : 0);
-    const long long L2 = (long long)p.tiles * cnt2;
-    const int np = 1 + int(boundaries_in((long long)tile * cnt2, (long long)(tile + 1) * cnt2 - 1, L2, p.P));
+    const int L2 = p.tiles * cnt2;
+    const int np = 1 + bnd_in(tile * cnt2, (tile + 1) * cnt2 - 1, L2, p.P);
     for (int o = 0; o < np && n < MAX_PIECES; ++o)
       out[n++] = uint32_t(((long long)tile * p.S + s2) * p.pmax + o);
   }
@@ -188,10 +219,13 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
 // and issue the MMAs for NTILE 8-column token tiles. MMA i of the step adds
 // into accumulator set i % (4 / NTILE): four independent chains per warp,
 // instead of sixteen MMAs serialised on one accumulator.
-template <int NTILE>
+// EARLY: after loading its share of the stage into registers the warp
+// releases the slot (lane 0 arrives on `empty`), so the refill overlaps the
+// decode and the MMAs.
+template <int NTILE, bool EARLY, bool PRED>
 __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* ss, int r, float (*acc)[4],
                                              const uint8_t* sx, const uint32_t* xcol, const bool* xon,
-                                             int kloc, int t) {
+                                             int kloc, int t, uint32_t empty_bar, int lane) {
   const int r1 = r + 8;
   // chunks 2t, 2t+1 of each row; the TMA 128-byte swizzle puts chunk c of row
   // r at position c ^ (r & 7)
@@ -201,6 +235,10 @@ __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* s
   const uint4 c11 = *reinterpret_cast<const uint4*>(sw + r1 * 128 + (((2 * t + 1) ^ (r1 & 7)) << 4));
   const uint32_t s0 = *reinterpret_cast<const uint32_t*>(ss + r * 16 + 4 * t);
   const uint32_t s1 = *reinterpret_cast<const uint32_t*>(ss + r1 * 16 + 4 * t);
+  if (EARLY) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar);
+  }
   const uint32_t w0[8] = {c00.x, c00.y, c00.z, c00.w, c01.x, c01.y, c01.z, c01.w};
   const uint32_t w1[8] = {c10.x, c10.y, c10.z, c10.w, c11.x, c11.y, c11.z, c11.w};
   // each scale byte duplicated, then converted: f16x2 {s, s}
@@ -229,7 +267,7 @@ __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* s
 #pragma unroll
       for (int nt = 0; nt < NTILE; ++nt) {
         uint2 bb = make_uint2(0u, 0u);
-        if (xon[nt]) bb = *reinterpret_cast<const uint2*>(sx + (xcol[nt] + xg) + 8 * i);
+        if (!PRED || xon[nt]) bb = *reinterpret_cast<const uint2*>(sx + (xcol[nt] + xg) + 8 * i);
         mma16816(acc[(i % NSET) * NTILE + nt], a0, a1, a2, a3, bb.x, bb.y);
       }
     }
@@ -241,12 +279,13 @@ __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* s
 // one tile; 2: hi + lo tiles, or two hi tiles; 4: two hi + two lo tiles).
 // Pieces of split tiles are written to the workspace and handed to the
 // settler warp through the queue (mbarriers q_full / q_empty).
-template <int MC, int NTILE>
+template <int MC, int NTILE, bool LO>
 __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* sS, const uint8_t* sX,
                                         const int* emax, uint32_t b_full, uint32_t b_empty,
                                         uint32_t b_qfull, uint32_t b_qempty,
-                                        volatile int* abort_flag, uint32_t* skip, int s, int cnt,
-                                        int a, int b, int L, int cw, int lane) {
+                                        volatile int* abort_flag, uint32_t* skip,
+                                        const volatile uint32_t* pre_flag, const float* pre_buf, int s,
+                                        int cnt, int a, int b, int L, int cw, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int r = 16 * cw + g;                           // row of the tile (and r + 8)
   int tok[4];
@@ -270,18 +309,24 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
   }
   const float gs = *p.gs;
   // X column of each token tile for this lane (B column g); shared memory
-  // holds only the 2M used columns: hi plane tokens 0..M-1, then lo plane
+  // holds only the 2M used columns: hi plane tokens 0..M-1, then lo plane.
+  // LO: some lo element is nonzero, lanes of absent tokens skip their loads
+  // (B = 0); otherwise the lo plane is all zero, the M <= 8 and M <= 16
+  // classes issue hi tiles only, and absent tokens read lo column 0 (zeros)
+  // so no load is predicated.
   uint32_t xcol[NTILE];
   bool xon[NTILE];
 #pragma unroll
   for (int nt = 0; nt < NTILE; ++nt) {
     int plane, tk;
     if (MC == 1) { plane = g >> 2; tk = g & 3; }
-    else if (MC == 2) { plane = nt; tk = g; }
-    else if (NTILE == 4) { plane = nt >> 1; tk = 8 * (nt & 1) + g; }
+    else if (MC == 2) { plane = LO ? nt : 0; tk = g; }
+    else if (LO) { plane = nt >> 1; tk = 8 * (nt & 1) + g; }
     else { plane = 0; tk = 8 * nt + g; }
-    xon[nt] = tk < p.M;
-    xcol[nt] = uint32_t(plane * p.M + (xon[nt] ? tk : 0)) * uint32_t(p.xstride);
+    const bool valid = tk < p.M;
+    xon[nt] = valid;
+    if (LO) xcol[nt] = uint32_t(plane * p.M + (valid ? tk : 0)) * uint32_t(p.xstride);
+    else xcol[nt] = uint32_t(valid ? plane * p.M + tk : p.M) * uint32_t(p.xstride);
   }
   float acc[4][4];
 #pragma unroll
@@ -291,12 +336,19 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
   int seg_start = a;
   int nsplit = 0;                                      // split segments handed to the settler
   int tile = a / cnt, j = a - tile * cnt;
+  const int pre_tile = MC == 1 ? prefetch_tile(p, a, b, cnt, L) : -1;
   for (int idx = a; idx < b; ++idx) {
     const bool ok = wait_bar(b_full + 8 * st, ph, abort_flag, p, ST_TIMEOUT_CONSUMER);
     if (!__all_sync(0xffffffffu, ok)) break;
-    compute_step<NTILE>(sW + st * W_BYTES, sS + st * S_BYTES, r, acc, sX, xcol, xon, j * KS, t);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(b_empty + 8 * st);
+    // the M <= 8 classes release the slot as soon as their share is in
+    // registers; the M <= 16 class has no registers to spare for that
+    constexpr bool EARLY = MC < 3;
+    compute_step<NTILE, EARLY, LO>(sW + st * W_BYTES, sS + st * S_BYTES, r, acc, sX, xcol, xon, j * KS, t,
+                               b_empty + 8 * st, lane);
+    if (!EARLY) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_empty + 8 * st);
+    }
     if (++st == p.nstage) { st = 0; ph ^= 1u; }
     const int jcur = j;
     const int tcur = tile;
@@ -336,8 +388,9 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     } else if (MC == 2) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        v[e][0] = at[0][e] * fh[e] + at[1][e] * fl[e];
-        v[e][1] = at[0][2 + e] * fh[e] + at[1][2 + e] * fl[e];
+        const float l0 = NTILE == 2 ? at[1 % NTILE][e] : 0.0f, l1 = NTILE == 2 ? at[1 % NTILE][2 + e] : 0.0f;
+        v[e][0] = at[0][e] * fh[e] + l0 * fl[e];
+        v[e][1] = at[0][2 + e] * fh[e] + l1 * fl[e];
       }
     } else {
 #pragma unroll
@@ -372,14 +425,29 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
                                 ST_TIMEOUT_CONSUMER);
       if (!__all_sync(0xffffffffu, okq)) break;
     }
-    const int ord = int(boundaries_in((long long)tcur * cnt, this_start, L, p.P));
+    const int ord = bnd_in(tcur * cnt, this_start, L, p.P);
     bool done_here = false;
-    if (p.S == 1 && ord == 0 && idx + 1 == b) {
+    if (MC == 1 && tcur == pre_tile && ord == 0 && idx + 1 == b &&
+        __all_sync(0xffffffffu, *pre_flag != 0u)) {
+      // the settler has copied the other piece into shared memory
+      __threadfence_block();
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int m = tok[e];
+        if (m >= 0 && m < p.M) {
+          if (row0 < p.N) p.y[size_t(m) * p.N + row0] = float_to_bf16_bits(gs * (v[e][0] + pre_buf[m * TROWS + r]));
+          if (row1 < p.N) p.y[size_t(m) * p.N + row1] = float_to_bf16_bits(gs * (v[e][1] + pre_buf[m * TROWS + r + 8]));
+        }
+      }
+      __syncwarp();
+      if (lane == 0) *reinterpret_cast<volatile uint32_t*>(p.counters + tcur * NCW + cw) = 0u;
+      done_here = true;
+    } else if (p.S == 1 && ord == 0 && idx + 1 == b) {
       // The CTA's last segment holds the tile's first k-range. The other
       // pieces were the first segments of the next CTAs and are usually
       // counted by now: then this warp adds them to its registers and stores
       // its rows without writing a partial.
-      const int np = 1 + int(boundaries_in((long long)tcur * cnt, (long long)(tcur + 1) * cnt - 1, L, p.P));
+      const int np = 1 + bnd_in(tcur * cnt, (tcur + 1) * cnt - 1, L, p.P);
       if (np - 1 <= FAST_MAX) {
         uint32_t* ctr = p.counters + tcur * NCW + cw;
         const uint32_t seen = ld_relaxed_gpu(ctr);
@@ -447,8 +515,9 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
 // itself.
 __device__ __forceinline__ void settle(const Params& p, uint32_t b_qfull, uint32_t b_qempty,
                                        volatile int* abort_flag, uint32_t* skip, uint32_t* list,
-                                       uint32_t* nlist, uint32_t* pieces, int cnt, int a, int b,
-                                       int lane) {
+                                       uint32_t* nlist, uint32_t* pieces, volatile uint32_t* pre_flag,
+                                       float* pre_buf, int cnt, int a, int b, int L, int lane) {
+  const int pre_tile = prefetch_tile(p, a, b, cnt, L);
   int nsplit = 0;
   int seg_start = a;
   int tile = a / cnt, j = a - tile * cnt;
@@ -461,14 +530,37 @@ __device__ __forceinline__ void settle(const Params& p, uint32_t b_qfull, uint32
     const bool whole = (p.S == 1) && (this_start == tcur * cnt) && (jcur + 1 == cnt);
     if (whole) continue;
     const int qs = nsplit % QN;
-    const bool ok = wait_bar(b_qfull + 8 * qs, uint32_t(nsplit / QN) & 1u, abort_flag, p, ST_TIMEOUT_SETTLER);
+    const uint32_t qpar = uint32_t(nsplit / QN) & 1u;
+    if (tcur == pre_tile && idx + 1 == b) {
+      // While the consumers work on the last piece: if the other piece of
+      // this tile (the next CTA's first segment) gets counted on every row
+      // group first, copy it into shared memory for the consumers.
+      bool copied = false;
+      const long long t0 = clock64();
+      while (!__any_sync(0xffffffffu, mbar_test(b_qfull + 8 * qs, qpar))) {
+        if (!copied) {
+          const bool ready = lane >= NCW || ld_acquire_gpu(p.counters + tcur * NCW + lane) == 1u;
+          if (__all_sync(0xffffffffu, ready)) {
+            const float* part = p.partials + ((long long)tcur * p.pmax + 1) * p.M * TROWS;
+            for (int u = lane; u < p.M * TROWS; u += 32) pre_buf[u] = __ldcg(part + u);
+            __syncwarp();
+            __threadfence_block();
+            if (lane == 0) *pre_flag = 1u;
+            copied = true;
+          }
+        }
+        if (*abort_flag || clock64() - t0 > p.timeout) break;   // wait_bar below reports it
+        __nanosleep(200);
+      }
+    }
+    const bool ok = wait_bar(b_qfull + 8 * qs, qpar, abort_flag, p, ST_TIMEOUT_SETTLER, 20000);
     if (!__all_sync(0xffffffffu, ok)) return;
     // total pieces of the tile over all slices
     int npieces = 0;
     for (int s2 = 0; s2 < p.S; ++s2) {
       const int cnt2 = p.ks_base + (s2 < p.ks_rem ? 1 : 0);
-      const long long L2 = (long long)p.tiles * cnt2;
-      npieces += 1 + int(boundaries_in((long long)tcur * cnt2, (long long)(tcur + 1) * cnt2 - 1, L2, p.P));
+      const int L2 = p.tiles * cnt2;
+      npieces += 1 + bnd_in(tcur * cnt2, (tcur + 1) * cnt2 - 1, L2, p.P);
     }
     const uint32_t sk = skip[qs];
     bool last = false;
@@ -520,6 +612,8 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
   uint32_t* skip = reinterpret_cast<uint32_t*>(misc + MISC_SKIP);    // [QN]
   uint32_t* pieces = reinterpret_cast<uint32_t*>(misc + MISC_PIECES);  // [MAX_PIECES + 1]
   uint32_t* list = reinterpret_cast<uint32_t*>(misc + MISC_LIST);    // [LIST_MAX][2]
+  volatile uint32_t* pre_flag = reinterpret_cast<volatile uint32_t*>(misc + MISC_PREFLAG);
+  float* pre_buf = reinterpret_cast<float*>(misc + MISC_PREBUF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(flags + 1);
   const uint32_t b_full = smem_u32(bars), b_empty = b_full + 8 * NSTAGE_MAX;
   const uint32_t b_qfull = b_empty + 8 * NSTAGE_MAX, b_qempty = b_qfull + 8 * QN;
@@ -539,6 +633,7 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     for (int i = 0; i < QN; ++i) { mbar_init(b_qfull + 8 * i, NCW); mbar_init(b_qempty + 8 * i, 1); }
     for (int m = 0; m < 16; ++m) emax[m] = INT_MIN;
     flags[0] = 0u; flags[1] = 0u; flags[2] = 0u;
+    *pre_flag = 0u;
     for (int i = 0; i < QN; ++i) skip[i] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -577,7 +672,7 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
   } else if (warp == WARP_SETTLE) {
     // ---------------------------------------------------------------- settler
     asm volatile("griddepcontrol.wait;" ::: "memory");   // counters of the previous grid
-    settle(p, b_qfull, b_qempty, abort_flag, skip, list, flags + 2, pieces, cnt, a, b, lane);
+    settle(p, b_qfull, b_qempty, abort_flag, skip, list, flags + 2, pieces, pre_flag, pre_buf, cnt, a, b, L, lane);
   } else {
     // ------------------------------------------------ consumers: stage X first
     // X, the global scale, Y and the workspace may belong to the previous grid
@@ -586,75 +681,85 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     constexpr int NCT = NCW * 32;
     const int chunks = klen / 8;
     const int nreal = p.M * chunks;
-    uint4 xv[MAXC];
+    // 1. X slice -> shared memory as raw bf16, in the hi plane's places, and
+    //    the per-token exponent maximum (lanes holding the same token reduce
+    //    in the warp: one shared-memory atomic per token and warp)
+    for (int base = ctid & ~31; base < nreal; base += 2 * NCT) {   // warp-uniform bound
+      uint4 xv[2];
+      int mm[2], kk[2];
 #pragma unroll
-    for (int cc = 0; cc < MAXC; ++cc) {
-      const int u = ctid + cc * NCT;
-      if (u < nreal) {
-        const int m = u / chunks, kc = u - m * chunks;
-        xv[cc] = *reinterpret_cast<const uint4*>(p.x + size_t(m) * p.K + k0e + 8 * kc);
-      }
-    }
-#pragma unroll
-    for (int cc = 0; cc < MAXC; ++cc) {
-      const int u = ctid + cc * NCT;
-      if (u < nreal) {
-        const int m = u / chunks;
-        const uint32_t w[4] = {xv[cc].x, xv[cc].y, xv[cc].z, xv[cc].w};
-        int mx = INT_MIN;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint32_t bb = (w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
-          if (bb & 0x7FFFu) { uint32_t sg; mx = max(mx, bf16_exp(bb, sg)); }
+      for (int h = 0; h < 2; ++h) {
+        const int u = base + (ctid & 31) + h * NCT;
+        mm[h] = -1;
+        if (u < nreal) {
+          mm[h] = u / chunks;
+          kk[h] = u - mm[h] * chunks;
+          xv[h] = *reinterpret_cast<const uint4*>(p.x + size_t(mm[h]) * p.K + k0e + 8 * kk[h]);
         }
-        if (mx != INT_MIN) atomicMax(&emax[m], mx);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        int mx = INT_MIN;
+        if (mm[h] >= 0) {
+          uint8_t* ch = sX + size_t(mm[h]) * p.xstride;
+          *reinterpret_cast<uint2*>(ch + x_off(8 * kk[h])) = make_uint2(xv[h].x, xv[h].y);
+          *reinterpret_cast<uint2*>(ch + x_off(8 * kk[h] + 4)) = make_uint2(xv[h].z, xv[h].w);
+          const uint32_t w[4] = {xv[h].x, xv[h].y, xv[h].z, xv[h].w};
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t bb = (w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
+            if (bb & 0x7FFFu) { uint32_t sg; mx = max(mx, bf16_exp(bb, sg)); }
+          }
+        }
+        const unsigned grp = __match_any_sync(0xffffffffu, mm[h]);
+        const int gmx = __reduce_max_sync(grp, mx);
+        if (mm[h] >= 0 && gmx != INT_MIN && (threadIdx.x & 31) == __ffs(grp) - 1) atomicMax(&emax[mm[h]], gmx);
       }
     }
     named_bar(BAR_CONSUMERS, NCT);
+    // 2. in place: raw bf16 -> hi plane, and the lo plane next to it
     bool lo_used = false;
+#pragma unroll 1
+    for (int u = ctid; u < nreal; u += NCT) {
+      const int m = u / chunks, kc = u - m * chunks;
+      const int sh = (emax[m] == INT_MIN) ? 0 : 14 - emax[m];
+      const uint32_t o0 = x_off(8 * kc), o1 = x_off(8 * kc + 4);
+      uint8_t* ch = sX + size_t(m) * p.xstride;
+      uint8_t* cl = sX + size_t(p.M + m) * p.xstride;
+      const uint2 r0 = *reinterpret_cast<const uint2*>(ch + o0), r1 = *reinterpret_cast<const uint2*>(ch + o1);
+      const uint32_t w[4] = {r0.x, r0.y, r1.x, r1.y};
+      uint32_t hi[4] = {0u, 0u, 0u, 0u}, lo[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int cc = 0; cc < MAXC; ++cc) {
-      const int u = ctid + cc * NCT;
-      if (u < nreal) {
-        const int m = u / chunks, kc = u - m * chunks;
-        const int sh = (emax[m] == INT_MIN) ? 0 : 14 - emax[m];
-        const uint32_t w[4] = {xv[cc].x, xv[cc].y, xv[cc].z, xv[cc].w};
-        uint32_t hi[4] = {0u, 0u, 0u, 0u}, lo[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint32_t bb = (w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
-          if (bb & 0x7FFFu) {
-            uint32_t sg;
-            const int th = bf16_exp(bb, sg) + sh;
-            if (th >= -14) hi[q >> 1] |= make_f16(bb >> 15, th, sg) << (16 * (q & 1));
-            else lo[q >> 1] |= make_f16(bb >> 15, th + LO_SHIFT, sg) << (16 * (q & 1));
-          }
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t bb = (w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
+        if (bb & 0x7FFFu) {
+          uint32_t sg;
+          const int th = bf16_exp(bb, sg) + sh;
+          if (th >= -14) hi[q >> 1] |= make_f16(bb >> 15, th, sg) << (16 * (q & 1));
+          else lo[q >> 1] |= make_f16(bb >> 15, th + LO_SHIFT, sg) << (16 * (q & 1));
         }
-        lo_used |= (lo[0] | lo[1] | lo[2] | lo[3]) != 0u;
-        const uint32_t o0 = x_off(8 * kc), o1 = x_off(8 * kc + 4);
-        uint8_t* ch = sX + size_t(m) * p.xstride;
-        uint8_t* cl = sX + size_t(p.M + m) * p.xstride;
-        *reinterpret_cast<uint2*>(ch + o0) = make_uint2(hi[0], hi[1]);
-        *reinterpret_cast<uint2*>(ch + o1) = make_uint2(hi[2], hi[3]);
-        *reinterpret_cast<uint2*>(cl + o0) = make_uint2(lo[0], lo[1]);
-        *reinterpret_cast<uint2*>(cl + o1) = make_uint2(lo[2], lo[3]);
       }
+      lo_used |= (lo[0] | lo[1] | lo[2] | lo[3]) != 0u;
+      *reinterpret_cast<uint2*>(ch + o0) = make_uint2(hi[0], hi[1]);
+      *reinterpret_cast<uint2*>(ch + o1) = make_uint2(hi[2], hi[3]);
+      *reinterpret_cast<uint2*>(cl + o0) = make_uint2(lo[0], lo[1]);
+      *reinterpret_cast<uint2*>(cl + o1) = make_uint2(lo[2], lo[3]);
     }
     if (lo_used) atomicOr(&flags[0], 1u);
     named_bar(BAR_CONSUMERS, NCT);
     const bool need_lo = flags[0] != 0u;
 
     const int cw = warp - 1;
+#define NVFP4_CONSUME(MC_, NT_, LO_) \
+  consume<MC_, NT_, LO_>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, pre_flag, pre_buf, s, cnt, a, b, L, cw, lane)
     if (MC == 1) {
-      consume<1, 1>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, s, cnt, a, b, L, cw, lane);
+      if (need_lo) NVFP4_CONSUME(1, 1, true); else NVFP4_CONSUME(1, 1, false);
     } else if (MC == 2) {
-      consume<2, 2>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, s, cnt, a, b, L, cw, lane);
+      if (need_lo) NVFP4_CONSUME(2, 2, true); else NVFP4_CONSUME(2, 1, false);
     } else {
-      if (need_lo)
-        consume<3, 4>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, s, cnt, a, b, L, cw, lane);
-      else
-        consume<3, 2>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, s, cnt, a, b, L, cw, lane);
+      if (need_lo) NVFP4_CONSUME(3, 4, true); else NVFP4_CONSUME(3, 2, false);
     }
+#undef NVFP4_CONSUME
   }
   __syncthreads();
   // ------------------------------------------------------------- end phase
@@ -686,8 +791,7 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   c.tiles = (c.N + TROWS - 1) / TROWS;
   const int ksteps = c.K / KS;
   const long long x_budget = (long long)optin - 1024 - (long long)NSTAGE_MIN * STAGE_BYTES - MISC_BYTES;
-  // largest slice (in steps) whose two X planes fit next to the ring and whose
-  // chunks the consumers hold in registers (M * steps * KS / 8 <= MAXC * consumer threads)
+  // largest slice (in steps) whose two X planes fit next to the ring;
   // column stride: the padded groups, rounded to 32 mod 128 bytes so that
   // columns g and g+1 start 8 banks apart
   auto stride_for = [](int ks) {
@@ -695,8 +799,7 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
     return ((base - 32 + 127) / 128) * 128 + 32;
   };
   auto fits = [&](int ks) {
-    return (long long)c.ncols * stride_for(ks) <= x_budget &&
-           (long long)c.M * ks * KS / 8 <= (long long)MAXC * NCW * 32;
+    return (long long)c.ncols * stride_for(ks) <= x_budget;
   };
   if (!fits(1)) return cudaErrorInvalidConfiguration;
   int max_ks = 1;
@@ -725,6 +828,8 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   }
   c.pmax = pmax;
   c.split = split;
+  // device-side piece arithmetic is 32-bit: (units + 1) * P must fit
+  if (((long long)c.tiles * (ks_base + 1) + 1) * P >= (1LL << 31)) return cudaErrorInvalidConfiguration;
   if ((long long)S * pmax > MAX_PIECES) return cudaErrorInvalidConfiguration;
   {
     const long long left = (long long)optin - 1024 - (long long)c.ncols * c.xstride - MISC_BYTES;

@@ -108,6 +108,17 @@ __device__ __forceinline__ bool mbar_test(uint32_t b, uint32_t parity) {
       : "=r"(ok) : "r"(b), "r"(parity) : "memory");
   return ok != 0;
 }
+// Same probe, but the thread may sleep in hardware until the phase completes
+// or about `hint_ns` nanoseconds pass, instead of spinning on the barrier.
+__device__ __forceinline__ bool mbar_wait_hint(uint32_t b, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(b), "r"(parity), "r"(hint_ns) : "memory");
+  return ok != 0;
+}
 // 2D tiled TMA load into shared memory, completing on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y,
                                             uint32_t bar) {
