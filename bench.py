@@ -349,6 +349,26 @@ def cpu_baseline(sample_rows: int = 34816, M: int = 1):
                       "median of 3" % (M, wl.K, rows, wl.N)}
 
 
+def measured_traffic(variant: str, workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    record (profiles/traffic.json), or None when the kernel's sources have
+    changed since the capture or the capture was of another workload."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    kernel = {"mma": "k_mma"}.get(variant)
+    if kernel is None or not os.path.exists(path):
+        return None
+    rec = json.load(open(path)).get(kernel)
+    if not rec or rec.get("workload") != workload:
+        return None
+    h = hashlib.sha256()
+    for f in rec["sources"]:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if h.hexdigest() != rec["sources_sha256"]:
+        return None
+    return rec["traffic_bytes_per_launch"]
+
+
 def run_ours(args):
     import torch
     world, rank, local = dist_setup(args.gpus)
@@ -412,7 +432,10 @@ def run_ours(args):
             "pct_of_measured_peak": 100 * per_gpu / peak,
             "pct_of_nominal_8TBps": 100 * per_gpu / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s",
-                         "frac": per_gpu / peak, "traffic": None,
+                         "frac": per_gpu / peak,
+                         "traffic": measured_traffic(["auto", "gemv", "mma", "tc"][pb.variant],
+                                                     "%s projection M=%d K=%d N=%d" %
+                                                     (args.workload, pb.M, pb.K, pb.N)),
                          "peak_kind": peak_kind + " device-copy bandwidth (MEASURED_PEAKS hbm_gbs)"},
             "gpu_launches": launches,
             "clocks": clocks,

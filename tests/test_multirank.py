@@ -66,3 +66,13 @@ def test_bytes_per_call_matches_oracle_model():
     import oracle
     for M, N, K in [(1, 34816, 5120), (16, 34816, 5120), (4, 5120, 17408), (8, 248320, 5120)]:
         assert bench.bytes_per_call(M, N, K) == oracle.bytes_model(M, N, K)
+
+
+def test_bench_traffic_record_matches_current_kernel_sources():
+    """The roofline traffic comes from a committed ncu record that is only
+    used while the kernel's sources are unchanged."""
+    import bench
+    t = bench.measured_traffic("mma", "decode projection M=1 K=5120 N=34816")
+    assert t is None or 100e6 < t < 120e6
+    assert bench.measured_traffic("mma", "some other workload") is None
+    assert bench.measured_traffic("tc", "decode projection M=1 K=5120 N=34816") is None
