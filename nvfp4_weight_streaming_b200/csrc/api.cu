@@ -40,6 +40,10 @@ struct nvfp4_plan_s {
   std::mutex map_mu;
   MapEntry maps[kMapCache];
   int map_next = 0;
+  // mma variant with X in the ring: descriptor of the X planes in the last
+  // workspace seen (the planes live in the workspace)
+  const void* xmap_ws = nullptr;
+  CUtensorMap xmap;
 };
 
 namespace {
@@ -241,7 +245,21 @@ nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
         if (!lookup_maps(plan, w_packed, w_scales, &mw, &ms)) return NVFP4_ERR_CUDA;
         const bool stall = (plan->flags & NVFP4_PLAN_TEST_STALL) != 0;
         const bool pdl = (plan->flags & NVFP4_PLAN_PDL) != 0;
-        e = nvfp4::launch_mma(plan->mma, &mw, &ms, w_global, xb, yb, workspace,
+        CUtensorMap mx;
+        if (plan->mma.xr) {
+          std::lock_guard<std::mutex> g(plan->map_mu);
+          if (plan->xmap_ws != workspace) {
+            const uint8_t* planes = static_cast<const uint8_t*>(workspace) + plan->mma.ws_x_off;
+            if (!nvfp4::encode_x_planes_map(planes, plan->mma.x_pitch, plan->mma.ncols, plan->mma.x_box,
+                                            &plan->xmap)) {
+              plan->xmap_ws = nullptr;
+              return NVFP4_ERR_CUDA;
+            }
+            plan->xmap_ws = workspace;
+          }
+          mx = plan->xmap;
+        }
+        e = nvfp4::launch_mma(plan->mma, &mw, &ms, &mx, w_global, xb, yb, workspace,
                               stall ? kStallTimeoutCycles : kTimeoutCycles, stall, pdl, st);
         break;
       }

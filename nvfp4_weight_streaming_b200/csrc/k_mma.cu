@@ -84,6 +84,9 @@ constexpr uint32_t ST_TIMEOUT_PRODUCER = 1u, ST_TIMEOUT_CONSUMER = 2u, ST_TIMEOU
 
 struct Params {
   int M, N, K, tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, nstage;
+  int xbytes, xbox_words, xbox_bytes;        // X in the ring: stage area, words per column, box bytes
+  const int* xemax;                          // X in the ring: per-token exponent maximum
+  const uint32_t* xlo;                       // X in the ring: per-token "lo plane used"
   const float* gs;
   const uint16_t* x;
   uint16_t* y;
@@ -219,13 +222,84 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
 // and issue the MMAs for NTILE 8-column token tiles. MMA i of the step adds
 // into accumulator set i % (4 / NTILE): four independent chains per warp,
 // instead of sixteen MMAs serialised on one accumulator.
+// Eight bf16 values (four words) -> their hi and lo f16 planes for the
+// token's shift sh (largest magnitude at 2^14; lo scaled by a further
+// 2^LO_SHIFT). Returns whether any lo element is nonzero.
+__device__ __forceinline__ bool x_split8(const uint32_t w[4], int sh, uint32_t hi[4], uint32_t lo[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) hi[q] = lo[q] = 0u;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const uint32_t bb = (w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
+    if (bb & 0x7FFFu) {
+      uint32_t sg;
+      const int th = bf16_exp(bb, sg) + sh;
+      if (th >= -14) hi[q >> 1] |= make_f16(bb >> 15, th, sg) << (16 * (q & 1));
+      else lo[q >> 1] |= make_f16(bb >> 15, th + LO_SHIFT, sg) << (16 * (q & 1));
+    }
+  }
+  return (lo[0] | lo[1] | lo[2] | lo[3]) != 0u;
+}
+
+// X in the ring: one CTA per token converts its row of X into the hi and lo
+// planes (columns m and M + m, `pitch` bytes each, the shared-memory group
+// layout of x_off) and records the token's exponent maximum and whether its
+// lo plane is used. The main kernel then loads one K-step of all planes per
+// ring stage.
+__global__ void __launch_bounds__(256)
+k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ planes, int pitch,
+        int* __restrict__ emax_out, uint32_t* __restrict__ lo_out) {
+  // X may be the previous grid's output; the main kernel may start now
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ int s_max[8];
+  const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint4* row = reinterpret_cast<const uint4*>(x + size_t(m) * K);
+  const int chunks = K / 8;
+  int mx = INT_MIN;
+  for (int kc = threadIdx.x; kc < chunks; kc += 256) {
+    const uint4 v = row[kc];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint32_t bb = (w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
+      if (bb & 0x7FFFu) { uint32_t sg; mx = max(mx, bf16_exp(bb, sg)); }
+    }
+  }
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (lane == 0) s_max[warp] = mx;
+  __syncthreads();
+  int emax = s_max[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) emax = max(emax, s_max[w]);
+  const int sh = emax == INT_MIN ? 0 : 14 - emax;
+  bool lo_used = false;
+  uint8_t* ch = planes + size_t(m) * pitch;
+  uint8_t* cl = planes + size_t(M + m) * pitch;
+  for (int kc = threadIdx.x; kc < chunks; kc += 256) {
+    const uint4 v = row[kc];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t hi[4], lo[4];
+    lo_used |= x_split8(w, sh, hi, lo);
+    *reinterpret_cast<uint2*>(ch + x_off(8 * kc)) = make_uint2(hi[0], hi[1]);
+    *reinterpret_cast<uint2*>(ch + x_off(8 * kc + 4)) = make_uint2(hi[2], hi[3]);
+    *reinterpret_cast<uint2*>(cl + x_off(8 * kc)) = make_uint2(lo[0], lo[1]);
+    *reinterpret_cast<uint2*>(cl + x_off(8 * kc + 4)) = make_uint2(lo[2], lo[3]);
+  }
+  lo_used = __syncthreads_or(lo_used);
+  if (threadIdx.x == 0) {
+    emax_out[m] = emax;
+    lo_out[m] = lo_used ? 1u : 0u;
+  }
+}
+
 // EARLY: after loading its share of the stage into registers the warp
 // releases the slot (lane 0 arrives on `empty`), so the refill overlaps the
 // decode and the MMAs.
 template <int NTILE, bool EARLY, bool PRED>
 __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* ss, int r, float (*acc)[4],
                                              const uint8_t* sx, const uint32_t* xcol, const bool* xon,
-                                             int kloc, int t, uint32_t empty_bar, int lane) {
+                                             uint32_t xg, int t, uint32_t empty_bar, int lane) {
   const int r1 = r + 8;
   // chunks 2t, 2t+1 of each row; the TMA 128-byte swizzle puts chunk c of row
   // r at position c ^ (r & 7)
@@ -248,8 +322,6 @@ __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* s
                            e4m3x2_to_f16x2(d0b >> 16)};
   const uint32_t sc1[4] = {e4m3x2_to_f16x2(d1a), e4m3x2_to_f16x2(d1a >> 16), e4m3x2_to_f16x2(d1b),
                            e4m3x2_to_f16x2(d1b >> 16)};
-  // lane t reads group 4 * (kloc / 256) + t of each X column
-  const uint32_t xg = uint32_t(XGROUP_BYTES * ((kloc >> 6) + t));
 #pragma unroll
   for (int wd = 0; wd < 8; ++wd) {
     uint32_t h0[4], h1[4];
@@ -279,7 +351,7 @@ __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* s
 // one tile; 2: hi + lo tiles, or two hi tiles; 4: two hi + two lo tiles).
 // Pieces of split tiles are written to the workspace and handed to the
 // settler warp through the queue (mbarriers q_full / q_empty).
-template <int MC, int NTILE, bool LO>
+template <int MC, int NTILE, bool LO, bool XR>
 __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* sS, const uint8_t* sX,
                                         const int* emax, uint32_t b_full, uint32_t b_empty,
                                         uint32_t b_qfull, uint32_t b_qempty,
@@ -325,8 +397,10 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     else { plane = 0; tk = 8 * nt + g; }
     const bool valid = tk < p.M;
     xon[nt] = valid;
-    if (LO) xcol[nt] = uint32_t(plane * p.M + (valid ? tk : 0)) * uint32_t(p.xstride);
-    else xcol[nt] = uint32_t(valid ? plane * p.M + tk : p.M) * uint32_t(p.xstride);
+    // column stride: the slice's column (staged X) or one K-step box (X in the ring)
+    const uint32_t cstride = XR ? uint32_t(p.xbox_words * 4) : uint32_t(p.xstride);
+    if (LO) xcol[nt] = uint32_t(plane * p.M + (valid ? tk : 0)) * cstride;
+    else xcol[nt] = uint32_t(valid ? plane * p.M + tk : p.M) * cstride;
   }
   float acc[4][4];
 #pragma unroll
@@ -343,8 +417,11 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     // the M <= 8 classes release the slot as soon as their share is in
     // registers; the M <= 16 class has no registers to spare for that
     constexpr bool EARLY = MC < 3;
-    compute_step<NTILE, EARLY, LO>(sW + st * W_BYTES, sS + st * S_BYTES, r, acc, sX, xcol, xon, j * KS, t,
-                               b_empty + 8 * st, lane);
+    // lane t reads 64-element group t of this step (staged X: of the slice)
+    const uint32_t xg = uint32_t(XGROUP_BYTES * (XR ? t : 4 * j + t));
+    compute_step<NTILE, EARLY, LO>(sW + st * W_BYTES, sS + st * S_BYTES, r, acc,
+                                   XR ? sX + st * p.xbytes : sX, xcol, xon, xg, t,
+                                   b_empty + 8 * st, lane);
     if (!EARLY) {
       __syncwarp();
       if (lane == 0) mbar_arrive(b_empty + 8 * st);
@@ -595,17 +672,21 @@ __device__ __forceinline__ void settle(const Params& p, uint32_t b_qfull, uint32
   }
 }
 
-template <int MC>
+// XR: X in the ring. Each stage also carries one K-step of the X planes
+// (prepared by k_xprep in the workspace), there are no K-slices and no
+// staging; otherwise the CTA stages its K-slice of X in shared memory.
+template <int MC, bool XR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s, const Params p) {
+k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
+      const __grid_constant__ CUtensorMap tm_x, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int nst = p.nstage;
   uint8_t* sW = smem;                                     // nst x 32 KB (1024-aligned)
   uint8_t* sS = smem + nst * W_BYTES;                     // nst x 4 KB
-  uint8_t* sX = sS + nst * S_BYTES;
-  uint8_t* misc = sX + size_t(p.ncols) * p.xstride;
+  uint8_t* sX = sS + nst * S_BYTES;                       // staged slice, or nst X boxes
+  uint8_t* misc = sX + (XR ? size_t(nst) * p.xbytes : size_t(p.ncols) * p.xstride);
   uint64_t* bars = reinterpret_cast<uint64_t*>(misc);     // full[8] empty[8] qfull[8] qempty[8]
   int* emax = reinterpret_cast<int*>(misc + MISC_EMAX);   // [16]
   uint32_t* flags = reinterpret_cast<uint32_t*>(misc + MISC_FLAGS);  // [0] need_lo [1] abort [2] list count
@@ -646,18 +727,43 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     if (lane == 0) {
       int n_issued = 0;
       const uint64_t pol = l2_evict_first_policy();
+      // XR: the first stages' weights go out before the previous grid has
+      // completed; their X boxes (written by k_xprep) only after it
+      const int pre_n = XR ? min(nst, b - a) : 0;
+      bool x_first = !XR;
       if (!p.stall) {
         int tile = a / cnt, j = a - tile * cnt, st = 0;
         uint32_t ph = 0;
         for (int idx = a; idx < b; ++idx, ++n_issued) {
+          if (!x_first && n_issued == pre_n) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            int j2 = a % cnt;
+            for (int n = 0; n < pre_n; ++n) {
+              tma_load_2d(smem_u32(sX + n * p.xbytes), &tm_x, (ks0 + j2) * p.xbox_words, 0, b_full + 8 * n);
+              if (++j2 == cnt) j2 = 0;
+            }
+            x_first = true;
+          }
           if (!wait_bar(b_empty + 8 * st, ph ^ 1u, abort_flag, p, ST_TIMEOUT_PRODUCER)) break;
-          mbar_expect_tx(b_full + 8 * st, STAGE_BYTES);
+          // the X box delivers exactly xbox_bytes (2M columns of one K-step)
+          mbar_expect_tx(b_full + 8 * st, STAGE_BYTES + (XR ? p.xbox_bytes : 0));
           tma_load_2d_hint(smem_u32(sW + st * W_BYTES), &tm_w, (ks0 + j) * (KS / 2), tile * TROWS,
                            b_full + 8 * st, pol);
           tma_load_2d_hint(smem_u32(sS + st * S_BYTES), &tm_s, (ks0 + j) * (KS / 16), tile * TROWS,
                            b_full + 8 * st, pol);
+          if (XR && x_first)
+            tma_load_2d(smem_u32(sX + st * p.xbytes), &tm_x, (ks0 + j) * p.xbox_words, 0, b_full + 8 * st);
           if (++j == cnt) { j = 0; ++tile; }
           if (++st == nst) { st = 0; ph ^= 1u; }
+        }
+        if (!x_first && n_issued == pre_n) {
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          int j2 = a % cnt;
+          for (int n = 0; n < pre_n; ++n) {
+            tma_load_2d(smem_u32(sX + n * p.xbytes), &tm_x, (ks0 + j2) * p.xbox_words, 0, b_full + 8 * n);
+            if (++j2 == cnt) j2 = 0;
+          }
+          x_first = true;
         }
       }
       if (*abort_flag) {
@@ -677,6 +783,19 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     // ------------------------------------------------ consumers: stage X first
     // X, the global scale, Y and the workspace may belong to the previous grid
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int cw = warp - 1;
+#define NVFP4_CONSUME(MC_, NT_, LO_, XR_, EMAX_) \
+  consume<MC_, NT_, LO_, XR_>(p, sW, sS, sX, EMAX_, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, pre_flag, pre_buf, s, cnt, a, b, L, cw, lane)
+    if constexpr (XR) {
+      // X arrives with the weights; exponents and lo flags come from k_xprep
+      bool need_lo = false;
+      for (int m = 0; m < p.M; ++m) need_lo |= p.xlo[m] != 0u;
+      if constexpr (MC == 2) {
+        if (need_lo) NVFP4_CONSUME(2, 2, true, true, p.xemax); else NVFP4_CONSUME(2, 1, false, true, p.xemax);
+      } else if constexpr (MC == 3) {
+        if (need_lo) NVFP4_CONSUME(3, 4, true, true, p.xemax); else NVFP4_CONSUME(3, 2, false, true, p.xemax);
+      }
+    } else {
     const int ctid = threadIdx.x - 32;                    // 0 .. NCW*32-1
     constexpr int NCT = NCW * 32;
     const int chunks = klen / 8;
@@ -728,18 +847,8 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
       uint8_t* cl = sX + size_t(p.M + m) * p.xstride;
       const uint2 r0 = *reinterpret_cast<const uint2*>(ch + o0), r1 = *reinterpret_cast<const uint2*>(ch + o1);
       const uint32_t w[4] = {r0.x, r0.y, r1.x, r1.y};
-      uint32_t hi[4] = {0u, 0u, 0u, 0u}, lo[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint32_t bb = (w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
-        if (bb & 0x7FFFu) {
-          uint32_t sg;
-          const int th = bf16_exp(bb, sg) + sh;
-          if (th >= -14) hi[q >> 1] |= make_f16(bb >> 15, th, sg) << (16 * (q & 1));
-          else lo[q >> 1] |= make_f16(bb >> 15, th + LO_SHIFT, sg) << (16 * (q & 1));
-        }
-      }
-      lo_used |= (lo[0] | lo[1] | lo[2] | lo[3]) != 0u;
+      uint32_t hi[4], lo[4];
+      lo_used |= x_split8(w, sh, hi, lo);
       *reinterpret_cast<uint2*>(ch + o0) = make_uint2(hi[0], hi[1]);
       *reinterpret_cast<uint2*>(ch + o1) = make_uint2(hi[2], hi[3]);
       *reinterpret_cast<uint2*>(cl + o0) = make_uint2(lo[0], lo[1]);
@@ -749,15 +858,13 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     named_bar(BAR_CONSUMERS, NCT);
     const bool need_lo = flags[0] != 0u;
 
-    const int cw = warp - 1;
-#define NVFP4_CONSUME(MC_, NT_, LO_) \
-  consume<MC_, NT_, LO_>(p, sW, sS, sX, emax, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, pre_flag, pre_buf, s, cnt, a, b, L, cw, lane)
-    if (MC == 1) {
-      if (need_lo) NVFP4_CONSUME(1, 1, true); else NVFP4_CONSUME(1, 1, false);
-    } else if (MC == 2) {
-      if (need_lo) NVFP4_CONSUME(2, 2, true); else NVFP4_CONSUME(2, 1, false);
+    if constexpr (MC == 1) {
+      if (need_lo) NVFP4_CONSUME(1, 1, true, false, emax); else NVFP4_CONSUME(1, 1, false, false, emax);
+    } else if constexpr (MC == 2) {
+      if (need_lo) NVFP4_CONSUME(2, 2, true, false, emax); else NVFP4_CONSUME(2, 1, false, false, emax);
     } else {
-      if (need_lo) NVFP4_CONSUME(3, 4, true); else NVFP4_CONSUME(3, 2, false);
+      if (need_lo) NVFP4_CONSUME(3, 4, true, false, emax); else NVFP4_CONSUME(3, 2, false, false, emax);
+    }
     }
 #undef NVFP4_CONSUME
   }
@@ -790,21 +897,30 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   c.ncols = 2 * c.M;                        // hi and lo plane of each token
   c.tiles = (c.N + TROWS - 1) / TROWS;
   const int ksteps = c.K / KS;
-  const long long x_budget = (long long)optin - 1024 - (long long)NSTAGE_MIN * STAGE_BYTES - MISC_BYTES;
-  // largest slice (in steps) whose two X planes fit next to the ring;
-  // column stride: the padded groups, rounded to 32 mod 128 bytes so that
-  // columns g and g+1 start 8 banks apart
+  // Column stride of a staged X slice: the padded groups, rounded to 32 mod
+  // 128 bytes so that columns g and g+1 start 8 banks apart. A K-step box of
+  // the X planes (X in the ring) is 4 groups = 544 bytes, also 32 mod 128.
   auto stride_for = [](int ks) {
     const int base = XGROUP_BYTES * (ks * KS / 64);
     return ((base - 32 + 127) / 128) * 128 + 32;
   };
-  auto fits = [&](int ks) {
-    return (long long)c.ncols * stride_for(ks) <= x_budget;
-  };
-  if (!fits(1)) return cudaErrorInvalidConfiguration;
-  int max_ks = 1;
-  while (max_ks < ksteps && fits(max_ks + 1)) ++max_ks;
-  const int S = (ksteps + max_ks - 1) / max_ks;
+  // M <= 4: the CTA stages its K-slice of X (2M columns) next to the ring.
+  // M > 4: 2M columns would force several K-slices; X goes through the ring.
+  c.xr = c.M > 4;
+  int S = 1;
+  if (c.xr) {
+    c.x_box = 4 * XGROUP_BYTES;
+    c.x_pitch = (c.K / 64) * XGROUP_BYTES;
+    c.xbytes = ((c.ncols * c.x_box + 127) / 128) * 128;
+  } else {
+    const long long x_budget = (long long)optin - 1024 - (long long)NSTAGE_MIN * STAGE_BYTES - MISC_BYTES;
+    auto fits = [&](int ks) { return (long long)c.ncols * stride_for(ks) <= x_budget; };
+    if (!fits(1)) return cudaErrorInvalidConfiguration;
+    int max_ks = 1;
+    while (max_ks < ksteps && fits(max_ks + 1)) ++max_ks;
+    S = (ksteps + max_ks - 1) / max_ks;
+    c.x_box = 0; c.x_pitch = 0; c.xbytes = 0;
+  }
   int P = num_sms / S;
   if (P < 1) return cudaErrorInvalidConfiguration;
   const int ks_base = ksteps / S, ks_rem = ksteps % S;
@@ -813,7 +929,7 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   c.S = S; c.P = P; c.ks_base = ks_base; c.ks_rem = ks_rem;
   c.grid = S * P;
   c.xk_max = (ks_base + (ks_rem ? 1 : 0)) * KS;
-  c.xstride = stride_for(c.xk_max / KS);
+  c.xstride = c.xr ? c.x_box : stride_for(c.xk_max / KS);
   int pmax = 1;
   bool split = S > 1;
   for (int s = 0; s < S; ++s) {
@@ -832,52 +948,82 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   if (((long long)c.tiles * (ks_base + 1) + 1) * P >= (1LL << 31)) return cudaErrorInvalidConfiguration;
   if ((long long)S * pmax > MAX_PIECES) return cudaErrorInvalidConfiguration;
   {
-    const long long left = (long long)optin - 1024 - (long long)c.ncols * c.xstride - MISC_BYTES;
-    int nst = int(left / STAGE_BYTES);
+    const long long x_smem = c.xr ? 0 : (long long)c.ncols * c.xstride;
+    const long long left = (long long)optin - 1024 - x_smem - MISC_BYTES;
+    int nst = int(left / (STAGE_BYTES + c.xbytes));
     c.nstage = nst < NSTAGE_MAX ? nst : NSTAGE_MAX;
   }
   if (c.nstage < NSTAGE_MIN) return cudaErrorInvalidConfiguration;
-  c.smem = 1024 + size_t(c.nstage) * STAGE_BYTES + size_t(c.ncols) * c.xstride + MISC_BYTES;
+  c.smem = 1024 + size_t(c.nstage) * (STAGE_BYTES + c.xbytes) +
+           (c.xr ? 0 : size_t(c.ncols) * c.xstride) + MISC_BYTES;
+  if (c.smem > size_t(optin)) return cudaErrorInvalidConfiguration;
+  // workspace: status word, per-(tile, row group) counters, partial sums,
+  // and for X in the ring the X planes plus per-token exponent and lo flag
   c.ws_counters_off = 256;
   c.ws_partials_off = c.ws_counters_off + ((size_t(c.tiles) * NCW * 4 + 255) / 256) * 256;
-  c.ws_bytes = split ? c.ws_partials_off + size_t(c.tiles) * S * pmax * c.M * TROWS * 4 : 256;
-  if (c.smem > size_t(optin)) return cudaErrorInvalidConfiguration;
-  e = cudaFuncSetAttribute(k_mma<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  const size_t partials_end = split ? c.ws_partials_off + size_t(c.tiles) * S * pmax * c.M * TROWS * 4
+                                    : (c.xr ? c.ws_partials_off : 256);
+  if (c.xr) {
+    c.ws_x_off = ((partials_end + 255) / 256) * 256;
+    c.ws_xmeta_off = c.ws_x_off + ((size_t(c.ncols) * c.x_pitch + 255) / 256) * 256;
+    c.ws_bytes = c.ws_xmeta_off + 128;
+  } else {
+    c.ws_x_off = c.ws_xmeta_off = 0;
+    c.ws_bytes = partials_end;
+  }
+  e = cudaFuncSetAttribute(k_mma<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   return e;
 }
 
-cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s, const float* gs,
-                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
-                       bool stall, bool pdl, cudaStream_t st) {
+cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s, const void* map_x,
+                       const float* gs, const uint16_t* x, uint16_t* y, void* workspace,
+                       long long timeout_cycles, bool stall, bool pdl, cudaStream_t st) {
   using namespace mm;
   Params p;
   p.M = c.M; p.N = c.N; p.K = c.K; p.tiles = c.tiles; p.S = c.S; p.P = c.P;
   p.ks_base = c.ks_base; p.ks_rem = c.ks_rem; p.ncols = c.ncols; p.xk_max = c.xk_max;
   p.xstride = c.xstride; p.pmax = c.pmax; p.nstage = c.nstage;
+  p.xbytes = c.xbytes; p.xbox_words = c.x_box / 4; p.xbox_bytes = c.ncols * c.x_box;
   p.gs = gs; p.x = x; p.y = y;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   p.status = reinterpret_cast<uint32_t*>(wsb);
   p.counters = reinterpret_cast<uint32_t*>(wsb + c.ws_counters_off);
   p.partials = c.split ? reinterpret_cast<float*>(wsb + c.ws_partials_off) : nullptr;
+  p.xemax = c.xr ? reinterpret_cast<const int*>(wsb + c.ws_xmeta_off) : nullptr;
+  p.xlo = c.xr ? reinterpret_cast<const uint32_t*>(wsb + c.ws_xmeta_off + 64) : nullptr;
   p.timeout = timeout_cycles;
   p.stall = stall ? 1 : 0;
   const CUtensorMap& mw = *static_cast<const CUtensorMap*>(map_w);
   const CUtensorMap& ms = *static_cast<const CUtensorMap*>(map_s);
+  const CUtensorMap& mx = c.xr ? *static_cast<const CUtensorMap*>(map_x) : mw;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  if (c.xr) {
+    cudaLaunchConfig_t pc = {};
+    pc.gridDim = dim3(c.M);
+    pc.blockDim = dim3(256);
+    pc.stream = st;
+    pc.attrs = attr;
+    pc.numAttrs = pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&pc, k_xprep, x, c.M, c.K, wsb + c.ws_x_off, c.x_pitch,
+                                       reinterpret_cast<int*>(wsb + c.ws_xmeta_off),
+                                       reinterpret_cast<uint32_t*>(wsb + c.ws_xmeta_off + 64));
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(c.grid);
   cfg.blockDim = dim3(NUM_THREADS);
   cfg.dynamicSmemBytes = c.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  if (c.M <= 4) return cudaLaunchKernelEx(&cfg, k_mma<1>, mw, ms, p);
-  if (c.M <= 8) return cudaLaunchKernelEx(&cfg, k_mma<2>, mw, ms, p);
-  return cudaLaunchKernelEx(&cfg, k_mma<3>, mw, ms, p);
+  // after k_xprep the dependency is always programmatic: k_mma waits for it in-kernel
+  cfg.numAttrs = (pdl || c.xr) ? 1 : 0;
+  if (c.M <= 4) return cudaLaunchKernelEx(&cfg, k_mma<1, false>, mw, ms, mx, p);
+  if (c.M <= 8) return cudaLaunchKernelEx(&cfg, k_mma<2, true>, mw, ms, mx, p);
+  return cudaLaunchKernelEx(&cfg, k_mma<3, true>, mw, ms, mx, p);
 }
 
 }  // namespace nvfp4

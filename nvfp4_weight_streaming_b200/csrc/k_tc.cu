@@ -664,6 +664,22 @@ bool encode_weight_maps(int N, int K, int box_rows, const uint8_t* wp, const uin
   return r == CUDA_SUCCESS;
 }
 
+bool encode_x_planes_map(const void* planes, int pitch_bytes, int cols, int box_bytes, void* map) {
+  auto fn = tc::encode_fn();
+  if (!fn) return false;
+  // f16 X planes in the workspace: `cols` columns of `pitch_bytes`, read as
+  // 32-bit words, one box = one K-step of every column
+  const cuuint64_t dim[2] = {cuuint64_t(pitch_bytes / 4), cuuint64_t(cols)};
+  const cuuint64_t str[1] = {cuuint64_t(pitch_bytes)};
+  const cuuint32_t box[2] = {cuuint32_t(box_bytes / 4), cuuint32_t(cols)};
+  const cuuint32_t one[2] = {1, 1};
+  const CUresult r = fn(static_cast<CUtensorMap*>(map), CU_TENSOR_MAP_DATA_TYPE_UINT32, 2,
+                        const_cast<void*>(planes), dim, str, box, one, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool tensor_maps_supported() { return tc::encode_fn() != nullptr; }
 
 cudaError_t launch_tc(const TcConfig& c, const void* map_w, const void* map_s, const float* gs,

@@ -44,6 +44,8 @@ cudaError_t tc_configure(TcConfig& c, int num_sms);
 bool encode_weight_maps(int N, int K, int box_rows, const uint8_t* wp, const uint8_t* ws,
                         void* map_w, void* map_s);
 bool tensor_maps_supported();
+// TMA descriptor of the f16 X planes the mma variant keeps in its workspace.
+bool encode_x_planes_map(const void* planes, int pitch_bytes, int cols, int box_bytes, void* map);
 cudaError_t launch_tc(const TcConfig& c, const void* map_w, const void* map_s, const float* gs,
                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
                       bool stall, cudaStream_t st);
@@ -53,12 +55,17 @@ struct MmaConfig {
   int M, N, K;
   int tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, nstage, grid;
   bool split;
+  // X in the ring (M > 4): X planes prepared once per call in the workspace
+  bool xr;
+  int x_pitch, x_box, xbytes;
+  size_t ws_x_off, ws_xmeta_off;
   size_t smem, ws_counters_off, ws_partials_off, ws_bytes;
 };
 cudaError_t mma_configure(MmaConfig& c, int num_sms);
-cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s, const float* gs,
-                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
-                       bool stall, bool pdl, cudaStream_t st);
+// map_x: descriptor of the X planes in `workspace` (encode_x_planes_map), used when c.xr.
+cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s, const void* map_x,
+                       const float* gs, const uint16_t* x, uint16_t* y, void* workspace,
+                       long long timeout_cycles, bool stall, bool pdl, cudaStream_t st);
 constexpr int kMmaTileRows = 256;
 
 }  // namespace nvfp4
