@@ -360,26 +360,13 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
                                         int cnt, int a, int b, int L, int cw, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int r = 16 * cw + g;                           // row of the tile (and r + 8)
-  int tok[4];
-  float fh[4], fl[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) { tok[e] = -1; fh[e] = fl[e] = 0.0f; }
-  if (MC == 1) {
-    if (t < 2) { tok[0] = 2 * t; tok[1] = 2 * t + 1; }
-  } else {
-    tok[0] = 2 * t; tok[1] = 2 * t + 1;
-    if (MC == 3) { tok[2] = 8 + 2 * t; tok[3] = 9 + 2 * t; }
-  }
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int m = tok[e];
-    if (m >= 0 && m < p.M && emax[m] != INT_MIN) {
-      const int sh = 14 - emax[m];
-      fh[e] = ldexpf(1.0f, -sh);
-      fl[e] = ldexpf(1.0f, -(sh + LO_SHIFT));
-    }
-  }
-  const float gs = *p.gs;
+  // tokens of this lane's accumulator values (columns 2t, 2t+1 of a tile):
+  // e = 0, 1 from the first token tile, e = 2, 3 from the second (M > 8)
+  auto tok = [t](int e) {
+    if (MC == 1) return (t < 2 && e < 2) ? 2 * t + e : -1;
+    if (e < 2) return 2 * t + e;
+    return MC == 3 ? 8 + 2 * t + (e - 2) : -1;
+  };
   // X column of each token tile for this lane (B column g); shared memory
   // holds only the 2M used columns: hi plane tokens 0..M-1, then lo plane.
   // LO: some lo element is nonzero, lanes of absent tokens skip their loads
@@ -414,9 +401,9 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
   for (int idx = a; idx < b; ++idx) {
     const bool ok = wait_bar(b_full + 8 * st, ph, abort_flag, p, ST_TIMEOUT_CONSUMER);
     if (!__all_sync(0xffffffffu, ok)) break;
-    // the M <= 8 classes release the slot as soon as their share is in
-    // registers; the M <= 16 class has no registers to spare for that
-    constexpr bool EARLY = MC < 3;
+    // release the slot as soon as this warp's share of the weights is in
+    // registers, unless X is read from the same slot during the MMAs
+    constexpr bool EARLY = !XR;
     // lane t reads 64-element group t of this step (staged X: of the slice)
     const uint32_t xg = uint32_t(XGROUP_BYTES * (XR ? t : 4 * j + t));
     compute_step<NTILE, EARLY, LO>(sW + st * W_BYTES, sS + st * S_BYTES, r, acc,
@@ -448,7 +435,20 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
       }
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.0f;
-    // per-token values of this lane: v[e][0] row r, v[e][1] row r+8
+    // per-token values of this lane: v[e][0] row r, v[e][1] row r+8; the
+    // planes' scales 2^-sh (hi) and 2^-(sh + LO_SHIFT) (lo) undone here
+    float fh[4], fl[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int m = tok(e);
+      fh[e] = fl[e] = 0.0f;
+      if (m >= 0 && m < p.M && emax[m] != INT_MIN) {
+        const int sh = 14 - emax[m];
+        fh[e] = ldexpf(1.0f, -sh);
+        fl[e] = ldexpf(1.0f, -(sh + LO_SHIFT));
+      }
+    }
+    const float gs = *p.gs;
     float v[4][2];
 #pragma unroll
     for (int e = 0; e < 4; ++e) v[e][0] = v[e][1] = 0.0f;
@@ -487,7 +487,7 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     if (whole) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int m = tok[e];
+        const int m = tok(e);
         if (m >= 0 && m < p.M) {
           if (row0 < p.N) p.y[size_t(m) * p.N + row0] = float_to_bf16_bits(gs * v[e][0]);
           if (row1 < p.N) p.y[size_t(m) * p.N + row1] = float_to_bf16_bits(gs * v[e][1]);
@@ -510,7 +510,7 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
       __threadfence_block();
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int m = tok[e];
+        const int m = tok(e);
         if (m >= 0 && m < p.M) {
           if (row0 < p.N) p.y[size_t(m) * p.N + row0] = float_to_bf16_bits(gs * (v[e][0] + pre_buf[m * TROWS + r]));
           if (row1 < p.N) p.y[size_t(m) * p.N + row1] = float_to_bf16_bits(gs * (v[e][1] + pre_buf[m * TROWS + r + 8]));
@@ -539,7 +539,7 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
               const float* part = p.partials + ((long long)tcur * p.pmax + o) * p.M * TROWS;
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const int m = tok[e];
+                const int m = tok(e);
                 if (m >= 0 && m < p.M) {
                   sum[e][0] += __ldcg(part + m * TROWS + r);
                   sum[e][1] += __ldcg(part + m * TROWS + r + 8);
@@ -549,7 +549,7 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int m = tok[e];
+            const int m = tok(e);
             if (m >= 0 && m < p.M) {
               if (row0 < p.N) p.y[size_t(m) * p.N + row0] = float_to_bf16_bits(gs * sum[e][0]);
               if (row1 < p.N) p.y[size_t(m) * p.N + row1] = float_to_bf16_bits(gs * sum[e][1]);
@@ -566,7 +566,7 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
       float* part = p.partials + slot * p.M * TROWS;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int m = tok[e];
+        const int m = tok(e);
         if (m >= 0 && m < p.M) {
           part[m * TROWS + r] = v[e][0];
           part[m * TROWS + r + 8] = v[e][1];

@@ -239,13 +239,16 @@ def test_linear_doubling_x_doubles_y_exactly():
         assert np.array_equal(2 * a, b), VNAME[v]
 
 
-def test_linear_deterministic_and_rows_independent():
+@pytest.mark.parametrize("M", [1, 8, 16])
+def test_linear_deterministic_and_rows_independent(M):
+    """Back-to-back calls on one workspace give bit-identical Y (also catches
+    a ring slot refilled while its data is still being read)."""
     packed, scales, gs = quantized("decode")
     w = Weights(packed, scales, gs)
-    X = synth.x_bf16(synth.WORKLOADS["verify"], 16)
-    for v in variants_for(16, w.N, w.K):
+    X = synth.x_bf16(synth.WORKLOADS["verify"], M)
+    for v in variants_for(M, w.N, w.K):
         y1, _, _ = run_linear(w, X, v)
-        y2, _, _ = run_linear(w, X, v, repeat=2)
+        y2, _, _ = run_linear(w, X, v, repeat=3)
         assert np.array_equal(y1, y2), VNAME[v]
 
 
