@@ -393,3 +393,53 @@ def test_verify_projection_full(M):
 @pytest.mark.parametrize("M", [1, 4, 8, 16])
 def test_down_projection_full(M):
     full_check("down", M)
+
+
+# ----- lm_head: N = 248,320 (1.27e9 weights) ------------------------------
+
+_lm = {}
+
+
+def lm_head_weights():
+    """The lm_head workload quantised by the oracle in row chunks (the fp32
+    matrix would take 5 GB): the global scale is the largest chunk scale
+    (amax / (6 * 448) is monotonic in amax), then each chunk is quantised
+    with it."""
+    if "w" not in _lm:
+        wl = synth.WORKLOADS["lm_head"]
+        ch = 16384
+        spans = [slice(r, min(r + ch, wl.N)) for r in range(0, wl.N, ch)]
+        gs = max(oracle.global_scale(synth.weights_f32(wl, rows=sp)) for sp in spans)
+        packed = np.empty((wl.N, wl.K // 2), np.uint8)
+        scales = np.empty((wl.N, wl.K // 16), np.uint8)
+        for sp in spans:
+            p, s = oracle.quantize_rows(synth.weights_f32(wl, rows=sp), gs)
+            packed[sp] = p
+            scales[sp] = s
+        _lm["w"] = (packed, scales, gs)
+    return _lm["w"]
+
+
+@pytest.mark.parametrize("M", [1, 8, 16])
+def test_lm_head_full_logits_and_argmax(M):
+    """Every logit within tolerance of the oracle, and per token the argmax
+    over all 248,320 logits: the GPU's index is the oracle's, or (a bf16 tie
+    or near-tie at the top) one whose exact logit is within tolerance of the
+    oracle's maximum."""
+    packed, scales, gs = lm_head_weights()
+    wl = synth.WORKLOADS["lm_head"]
+    if "dev" not in _lm:
+        _lm["dev"] = Weights(packed, scales, gs)
+    w = _lm["dev"]
+    X = synth.x_bf16(wl, M)
+    y_ref, ad = oracle.linear(packed, scales, gs, X, M, wl.N, wl.K)
+    tol = oracle.tolerance(y_ref, ad)
+    for v in variants_for(M, wl.N, wl.K):
+        y, ok, _ = run_linear(w, X, v)
+        assert ok, VNAME[v]
+        check_tolerance(y, y_ref, ad)
+        yg = oracle.bf16_bits_to_f64(y)
+        for m in range(M):
+            jg, jr = int(np.argmax(yg[m])), int(np.argmax(y_ref[m]))
+            assert jg == jr or y_ref[m, jr] - y_ref[m, jg] <= tol[m, jr] + tol[m, jg], \
+                (VNAME[v], m, jg, jr)
