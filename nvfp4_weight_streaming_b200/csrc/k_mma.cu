@@ -679,9 +679,11 @@ template <int MC, bool XR>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
       const __grid_constant__ CUtensorMap tm_x, const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment (128-byte swizzled TMA destinations) by an offset, so
+  // every derived pointer stays visibly in the shared window (32-bit shared
+  // addressing instead of generic loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int nst = p.nstage;
   uint8_t* sW = smem;                                     // nst x 32 KB (1024-aligned)
   uint8_t* sS = smem + nst * W_BYTES;                     // nst x 4 KB
