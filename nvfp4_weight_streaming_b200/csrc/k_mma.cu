@@ -70,7 +70,9 @@ constexpr int NSTAGE_MAX = 8;             // deeper rings use what X leaves free
 constexpr int W_BYTES = TROWS * KS / 2;    // 32768
 constexpr int S_BYTES = TROWS * KS / 16;   // 4096
 constexpr int STAGE_BYTES = W_BYTES + S_BYTES;
-constexpr int MISC_BYTES = 1024 + 4096;
+constexpr int MISC_BASE = 1024;            // barriers, flags, lists
+// misc area size: for M <= 4 plus the prefetched piece [M][TROWS] floats
+inline int misc_bytes(int M) { return MISC_BASE + (M <= 4 ? M * TROWS * 4 : 0); }
 // misc area: barriers [0,256) (full, empty, qfull, qempty: 8 each), emax [256,320),
 // flags [320,336) (need_lo, abort, list count), skip masks [336,368),
 // piece slots [384,640), end-phase list [640,896)
@@ -78,6 +80,7 @@ constexpr int MISC_EMAX = 256, MISC_FLAGS = 320, MISC_SKIP = 336, MISC_PREFLAG =
               MISC_LIST = 640, MISC_PREBUF = 1024;   // prefetched piece: [M <= 4][TROWS] floats
 constexpr int LO_SHIFT = 29;
 constexpr int BAR_CONSUMERS = 1;           // named barrier of the consumer warps
+constexpr int XR_MIN_M = 5;                // token counts from which X goes through the ring
 
 constexpr uint32_t ST_TIMEOUT_PRODUCER = 1u, ST_TIMEOUT_CONSUMER = 2u, ST_TIMEOUT_SETTLER = 4u,
                    ST_TIMEOUT_DRAIN = 16u;
@@ -792,7 +795,9 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
       // X arrives with the weights; exponents and lo flags come from k_xprep
       bool need_lo = false;
       for (int m = 0; m < p.M; ++m) need_lo |= p.xlo[m] != 0u;
-      if constexpr (MC == 2) {
+      if constexpr (MC == 1) {
+        if (need_lo) NVFP4_CONSUME(1, 1, true, true, p.xemax); else NVFP4_CONSUME(1, 1, false, true, p.xemax);
+      } else if constexpr (MC == 2) {
         if (need_lo) NVFP4_CONSUME(2, 2, true, true, p.xemax); else NVFP4_CONSUME(2, 1, false, true, p.xemax);
       } else if constexpr (MC == 3) {
         if (need_lo) NVFP4_CONSUME(3, 4, true, true, p.xemax); else NVFP4_CONSUME(3, 2, false, true, p.xemax);
@@ -906,16 +911,17 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
     const int base = XGROUP_BYTES * (ks * KS / 64);
     return ((base - 32 + 127) / 128) * 128 + 32;
   };
-  // M <= 4: the CTA stages its K-slice of X (2M columns) next to the ring.
-  // M > 4: 2M columns would force several K-slices; X goes through the ring.
-  c.xr = c.M > 4;
+  // Small M: the CTA stages its K-slice of X (2M columns) next to the ring.
+  // From XR_MIN_M: 2M columns would force several K-slices; X goes through
+  // the ring.
+  c.xr = c.M >= XR_MIN_M;
   int S = 1;
   if (c.xr) {
     c.x_box = 4 * XGROUP_BYTES;
     c.x_pitch = (c.K / 64) * XGROUP_BYTES;
     c.xbytes = ((c.ncols * c.x_box + 127) / 128) * 128;
   } else {
-    const long long x_budget = (long long)optin - 1024 - (long long)NSTAGE_MIN * STAGE_BYTES - MISC_BYTES;
+    const long long x_budget = (long long)optin - 1024 - (long long)NSTAGE_MIN * STAGE_BYTES - misc_bytes(c.M);
     auto fits = [&](int ks) { return (long long)c.ncols * stride_for(ks) <= x_budget; };
     if (!fits(1)) return cudaErrorInvalidConfiguration;
     int max_ks = 1;
@@ -951,13 +957,13 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   if ((long long)S * pmax > MAX_PIECES) return cudaErrorInvalidConfiguration;
   {
     const long long x_smem = c.xr ? 0 : (long long)c.ncols * c.xstride;
-    const long long left = (long long)optin - 1024 - x_smem - MISC_BYTES;
+    const long long left = (long long)optin - 1024 - x_smem - misc_bytes(c.M);
     int nst = int(left / (STAGE_BYTES + c.xbytes));
     c.nstage = nst < NSTAGE_MAX ? nst : NSTAGE_MAX;
   }
   if (c.nstage < NSTAGE_MIN) return cudaErrorInvalidConfiguration;
   c.smem = 1024 + size_t(c.nstage) * (STAGE_BYTES + c.xbytes) +
-           (c.xr ? 0 : size_t(c.ncols) * c.xstride) + MISC_BYTES;
+           (c.xr ? 0 : size_t(c.ncols) * c.xstride) + misc_bytes(c.M);
   if (c.smem > size_t(optin)) return cudaErrorInvalidConfiguration;
   // workspace: status word, per-(tile, row group) counters, partial sums,
   // and for X in the ring the X planes plus per-token exponent and lo flag
@@ -974,6 +980,7 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
     c.ws_bytes = partials_end;
   }
   e = cudaFuncSetAttribute(k_mma<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   return e;
@@ -1023,7 +1030,10 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
   cfg.attrs = attr;
   // after k_xprep the dependency is always programmatic: k_mma waits for it in-kernel
   cfg.numAttrs = (pdl || c.xr) ? 1 : 0;
-  if (c.M <= 4) return cudaLaunchKernelEx(&cfg, k_mma<1, false>, mw, ms, mx, p);
+  if (c.M <= 4) {
+    if (c.xr) return cudaLaunchKernelEx(&cfg, k_mma<1, true>, mw, ms, mx, p);
+    return cudaLaunchKernelEx(&cfg, k_mma<1, false>, mw, ms, mx, p);
+  }
   if (c.M <= 8) return cudaLaunchKernelEx(&cfg, k_mma<2, true>, mw, ms, mx, p);
   return cudaLaunchKernelEx(&cfg, k_mma<3, true>, mw, ms, mx, p);
 }

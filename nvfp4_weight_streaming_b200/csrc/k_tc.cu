@@ -212,9 +212,9 @@ __device__ __forceinline__ int pieces_in_slice(const Params& p, int t, int s) {
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
      const Params p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment by an offset: derived pointers stay in the shared window
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const Smem L = smem_layout(p.nb, p.xk_max);
   uint8_t* sW = smem + L.off_w;
   uint8_t* sS = smem + L.off_s;
