@@ -225,23 +225,50 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
 // and issue the MMAs for NTILE 8-column token tiles. MMA i of the step adds
 // into accumulator set i % (4 / NTILE): four independent chains per warp,
 // instead of sixteen MMAs serialised on one accumulator.
-// Eight bf16 values (four words) -> their hi and lo f16 planes for the
-// token's shift sh (largest magnitude at 2^14; lo scaled by a further
-// 2^LO_SHIFT). Returns whether any lo element is nonzero.
+// Largest bf16 magnitude (bits, sign cleared) among the eight values of a
+// 16-byte chunk, with one packed 16-bit max per pair.
+__device__ __forceinline__ uint32_t bf16_mag_max8(const uint4& v) {
+  const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                              __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+// Exponent floor(log2 |x|) of the bf16 magnitude `mag`; INT_MIN for zero.
+__device__ __forceinline__ int bf16_mag_exp(uint32_t mag) {
+  if (mag == 0u) return INT_MIN;
+  const uint32_t e8 = mag >> 7;
+  if (e8) return int(e8) - 127;
+  return (31 - __clz(int(mag & 0x7Fu))) - 133;     // subnormal
+}
+
+// Two bf16 values (one word) -> their hi f16 pair and lo f16 pair for the
+// token's shift: x * 2^sh (exact: the scale is applied as two powers of two
+// f1 * f2) rounded to f16 is the hi plane (exact for |x * 2^sh| >= 2^-14:
+// 8 significant bits), the exact remainder scaled by 2^LO_SHIFT is the lo
+// plane. Returns the lo pair.
+__device__ __forceinline__ uint32_t x_split2(uint32_t w, float f1, float f2, uint32_t& hi) {
+  const float s0 = (__uint_as_float(w << 16) * f1) * f2;
+  const float s1 = (__uint_as_float(w & 0xFFFF0000u) * f1) * f2;
+  const __half2 h = __floats2half2_rn(s0, s1);       // low half = element 0
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  const float2 hb = __half22float2(h);
+  constexpr float kLo = 536870912.0f;                 // 2^LO_SHIFT
+  const __half2 l = __floats2half2_rn((s0 - hb.x) * kLo, (s1 - hb.y) * kLo);
+  return *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Eight bf16 values (four words) -> hi and lo planes for the token's shift
+// sh (largest magnitude at 2^14); returns whether any lo element is nonzero.
 __device__ __forceinline__ bool x_split8(const uint32_t w[4], int sh, uint32_t hi[4], uint32_t lo[4]) {
+  static_assert(LO_SHIFT == 29, "kLo above is 2^29");
+  const float f1 = __int_as_float((127 + sh / 2) << 23), f2 = __int_as_float((127 + sh - sh / 2) << 23);
+  uint32_t any = 0u;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) hi[q] = lo[q] = 0u;
-#pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    const uint32_t bb = (w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
-    if (bb & 0x7FFFu) {
-      uint32_t sg;
-      const int th = bf16_exp(bb, sg) + sh;
-      if (th >= -14) hi[q >> 1] |= make_f16(bb >> 15, th, sg) << (16 * (q & 1));
-      else lo[q >> 1] |= make_f16(bb >> 15, th + LO_SHIFT, sg) << (16 * (q & 1));
-    }
+  for (int q = 0; q < 4; ++q) {
+    lo[q] = x_split2(w[q], f1, f2, hi[q]);
+    any |= lo[q] & 0x7FFF7FFFu;
   }
-  return (lo[0] | lo[1] | lo[2] | lo[3]) != 0u;
+  return any != 0u;
 }
 
 // X in the ring: one CTA per token converts its row of X into the hi and lo
@@ -259,17 +286,9 @@ k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ plan
   const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint4* row = reinterpret_cast<const uint4*>(x + size_t(m) * K);
   const int chunks = K / 8;
-  int mx = INT_MIN;
-  for (int kc = threadIdx.x; kc < chunks; kc += 256) {
-    const uint4 v = row[kc];
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const uint32_t bb = (w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
-      if (bb & 0x7FFFu) { uint32_t sg; mx = max(mx, bf16_exp(bb, sg)); }
-    }
-  }
-  mx = __reduce_max_sync(0xffffffffu, mx);
+  uint32_t mag = 0u;
+  for (int kc = threadIdx.x; kc < chunks; kc += 256) mag = max(mag, bf16_mag_max8(row[kc]));
+  int mx = bf16_mag_exp(__reduce_max_sync(0xffffffffu, mag));
   if (lane == 0) s_max[warp] = mx;
   __syncthreads();
   int emax = s_max[0];
@@ -825,20 +844,15 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
       }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        int mx = INT_MIN;
+        uint32_t mag = 0u;
         if (mm[h] >= 0) {
           uint8_t* ch = sX + size_t(mm[h]) * p.xstride;
           *reinterpret_cast<uint2*>(ch + x_off(8 * kk[h])) = make_uint2(xv[h].x, xv[h].y);
           *reinterpret_cast<uint2*>(ch + x_off(8 * kk[h] + 4)) = make_uint2(xv[h].z, xv[h].w);
-          const uint32_t w[4] = {xv[h].x, xv[h].y, xv[h].z, xv[h].w};
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint32_t bb = (w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu;
-            if (bb & 0x7FFFu) { uint32_t sg; mx = max(mx, bf16_exp(bb, sg)); }
-          }
+          mag = bf16_mag_max8(xv[h]);
         }
         const unsigned grp = __match_any_sync(0xffffffffu, mm[h]);
-        const int gmx = __reduce_max_sync(grp, mx);
+        const int gmx = bf16_mag_exp(__reduce_max_sync(grp, mag));
         if (mm[h] >= 0 && gmx != INT_MIN && (threadIdx.x & 31) == __ffs(grp) - 1) atomicMax(&emax[mm[h]], gmx);
       }
     }

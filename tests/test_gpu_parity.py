@@ -289,6 +289,25 @@ def test_pdl_chained_calls_read_the_previous_output(M):
         nv.nvfp4_linear_destroy(plan)
 
 
+def test_rows_of_y_depend_only_on_their_row_of_x():
+    """Row m of Y from an M=16 call against the M=1 call on row m alone: within
+    tolerance of each other's oracle values (required); how many rows are bit
+    identical is reported, not required (the token classes differ)."""
+    packed, scales, gs = quantized("decode")
+    w = Weights(packed, scales, gs)
+    X = synth.x_bf16(synth.WORKLOADS["verify"], 16)
+    rows = np.arange(0, w.N, 97)
+    y_ref, ad = oracle.linear(packed, scales, gs, X, 16, w.N, w.K, rows=rows)
+    y16, _, _ = run_linear(w, X)
+    same = 0
+    for m in (0, 5, 15):
+        y1, _, _ = run_linear(w, X[m:m + 1])
+        check_tolerance(y1[:, rows], y_ref[m:m + 1], ad[m:m + 1])
+        check_tolerance(y16[m:m + 1, rows], y_ref[m:m + 1], ad[m:m + 1])
+        same += int(np.array_equal(y1[0], y16[m]))
+    print("rows bit-identical between M=1 and M=16 calls: %d of 3" % same)
+
+
 def test_linear_k_zero_writes_zeros_and_n_zero_is_noop():
     w = Weights(np.zeros((8, 0), np.uint8), np.zeros((8, 0), np.uint8), 1.0)
     w.packed = torch.zeros(16, dtype=torch.uint8, device="cuda")
