@@ -423,9 +423,10 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
   for (int idx = a; idx < b; ++idx) {
     const bool ok = wait_bar(b_full + 8 * st, ph, abort_flag, p, ST_TIMEOUT_CONSUMER);
     if (!__all_sync(0xffffffffu, ok)) break;
-    // release the slot as soon as this warp's share of the weights is in
-    // registers, unless X is read from the same slot during the MMAs
-    constexpr bool EARLY = !XR;
+    // The slot is released after the MMAs. (Releasing it as soon as the
+    // weights are in registers measured ~2% slower at M = 1, and is not
+    // possible with X in the ring, which is read during the MMAs.)
+    constexpr bool EARLY = false;
     // lane t reads 64-element group t of this step (staged X: of the slice)
     const uint32_t xg = uint32_t(XGROUP_BYTES * (XR ? t : 4 * j + t));
     compute_step<NTILE, EARLY, LO>(sW + st * W_BYTES, sS + st * S_BYTES, r, acc,
