@@ -98,11 +98,12 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
                                nvfp4_plan_t* out);
 
 /* Device workspace bytes nvfp4_linear_run needs for this plan (status word,
- * per-tile counters and fp32 partials of tiles computed in several pieces),
- * 0 if none. Zero-fill it once before first use: after every successful run
- * its status word and counters are zero again, so it can be reused without
- * clearing (the partial area never needs clearing). Two runs in flight at the
- * same time must not share a workspace. */
+ * per-tile counters and fp32 partials of tiles computed in several pieces;
+ * for the mma variant with M >= 5 also X converted to two f16 planes), 0 if
+ * none. Zero-fill it once before first use: after every successful run its
+ * status word and counters are zero again, so it can be reused without
+ * clearing (the partial and X areas never need clearing). Two runs in flight
+ * at the same time must not share a workspace. */
 size_t nvfp4_linear_workspace_bytes(nvfp4_plan_t plan);
 
 /* Chosen variant (NVFP4_VARIANT_*) and split-K factor of a plan; -1 if null. */
