@@ -1,0 +1,73 @@
+"""The oracle's pins catch plausible mistakes: each mutant below is the
+oracle's source with one planted error (built into a temporary directory,
+never into the package), and at least one pin of tests/test_oracle_pins.py
+must fail against it. The unmutated oracle passes them all (that module).
+
+Runs on the CPU only; the GPU path is not involved."""
+import inspect
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import tests.test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "nvfp4_oracle.cpp")
+
+# name -> (text in the oracle source, replacement); each text occurs exactly once
+MUTANTS = {
+    "nibble order swapped when packing": (
+        "out[j / 2] = uint8_t(q0 | (q1 << 4));",
+        "out[j / 2] = uint8_t(q1 | (q0 << 4));"),
+    "wrong scale block index in the linear": (
+        "ora_e4m3_decode(scales[n * (K / 16) + k / 16]) * double(gs);",
+        "ora_e4m3_decode(scales[n * (K / 16) + k / 32]) * double(gs);"),
+    "E2M1 sign dropped": (
+        "double mag = (e == 0) ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, int(e) - 1);\n  return s ? -mag : mag;",
+        "double mag = (e == 0) ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, int(e) - 1);\n  return mag;"),
+    "block scale divides by 4 instead of 6": (
+        "float t = amax_b / 6.0f;",
+        "float t = amax_b / 4.0f;"),
+    "ties rounded away from zero": (
+        "return (lo % 2 == 0) ? lo : hi;",
+        "return hi;"),
+    "X indexed transposed": (
+        "double p = wrow[size_t(k)] * xm[k];",
+        "double p = wrow[size_t(k)] * x[size_t(k * M + m) % size_t(M * K)];"),
+    "last product of each row dropped": (
+        "for (int64_t k = 0; k < K; ++k) {\n          double p",
+        "for (int64_t k = 0; k < K - 1; ++k) {\n          double p"),
+}
+
+PIN_TESTS = [(name, fn) for name, fn in sorted(vars(pins).items())
+             if name.startswith("test_") and callable(fn) and not inspect.signature(fn).parameters]
+
+
+def _build_mutant(tmp_path, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, "mutation site must be unique: %r" % old
+    path = tmp_path / "nvfp4_oracle_mutant.cpp"
+    path.write_text(src.replace(old, new))
+    lib = tmp_path / "libnvfp4_oracle_mutant.so"
+    subprocess.run(["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-shared",
+                    "-fPIC", "-pthread", "-I", os.path.dirname(SRC), "-o", str(lib), str(path)],
+                   check=True)
+    return str(lib)
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(mutant, tmp_path, monkeypatch):
+    lib = _build_mutant(tmp_path, *MUTANTS[mutant])
+    monkeypatch.setattr(oracle, "build", lambda force=False: lib)
+    monkeypatch.setattr(oracle, "_lib", None)
+    caught = []
+    try:
+        for name, fn in PIN_TESTS:
+            try:
+                fn()
+            except Exception:            # an assertion or a rejected result
+                caught.append(name)
+    finally:
+        oracle._lib = None               # the next user reloads the real oracle
+    assert caught, "no pin fails for mutant: %s" % mutant
