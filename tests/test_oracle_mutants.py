@@ -1,7 +1,7 @@
 """The oracle's pins catch plausible mistakes: each mutant below is the
-oracle's source with one planted error (built into a temporary directory,
-never into the package), and at least one pin of tests/test_oracle_pins.py
-must fail against it. The unmutated oracle passes them all (that module).
+oracle's source with one planted error (built under the repository's
+git-ignored _build/ folder, never into the package), and at least one pin of
+tests/test_oracle_pins.py must fail against it. The unmutated oracle passes them all (that module).
 
 Runs on the CPU only; the GPU path is not involved."""
 import inspect
@@ -14,6 +14,7 @@ import oracle
 import tests.test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "nvfp4_oracle.cpp")
+BUILD = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "_build", "oracle_mutants")
 
 # name -> (text in the oracle source, replacement); each text occurs exactly once
 MUTANTS = {
@@ -44,12 +45,14 @@ PIN_TESTS = [(name, fn) for name, fn in sorted(vars(pins).items())
              if name.startswith("test_") and callable(fn) and not inspect.signature(fn).parameters]
 
 
-def _build_mutant(tmp_path, old, new):
+def _build_mutant(tag, old, new):
     src = open(SRC).read()
     assert src.count(old) == 1, "mutation site must be unique: %r" % old
-    path = tmp_path / "nvfp4_oracle_mutant.cpp"
-    path.write_text(src.replace(old, new))
-    lib = tmp_path / "libnvfp4_oracle_mutant.so"
+    os.makedirs(BUILD, exist_ok=True)
+    path = os.path.join(BUILD, "mutant_%s_%d.cpp" % (tag, os.getpid()))
+    with open(path, "w") as f:
+        f.write(src.replace(old, new))
+    lib = path[:-4] + ".so"
     subprocess.run(["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-shared",
                     "-fPIC", "-pthread", "-I", os.path.dirname(SRC), "-o", str(lib), str(path)],
                    check=True)
@@ -57,8 +60,8 @@ def _build_mutant(tmp_path, old, new):
 
 
 @pytest.mark.parametrize("mutant", sorted(MUTANTS))
-def test_pins_catch_planted_mistake(mutant, tmp_path, monkeypatch):
-    lib = _build_mutant(tmp_path, *MUTANTS[mutant])
+def test_pins_catch_planted_mistake(mutant, monkeypatch):
+    lib = _build_mutant("%d" % sorted(MUTANTS).index(mutant), *MUTANTS[mutant])
     monkeypatch.setattr(oracle, "build", lambda force=False: lib)
     monkeypatch.setattr(oracle, "_lib", None)
     caught = []
@@ -70,4 +73,7 @@ def test_pins_catch_planted_mistake(mutant, tmp_path, monkeypatch):
                 caught.append(name)
     finally:
         oracle._lib = None               # the next user reloads the real oracle
+        for f in (lib, lib[:-3] + ".cpp"):
+            if os.path.exists(f):
+                os.remove(f)
     assert caught, "no pin fails for mutant: %s" % mutant
