@@ -353,7 +353,6 @@ def measured_traffic(variant: str, workload: str):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     record (profiles/traffic.json), or None when the kernel's sources have
     changed since the capture or the capture was of another workload."""
-    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     kernel = {"mma": "k_mma"}.get(variant)
     if kernel is None or not os.path.exists(path):
@@ -361,12 +360,23 @@ def measured_traffic(variant: str, workload: str):
     rec = json.load(open(path)).get(kernel)
     if not rec or rec.get("workload") != workload:
         return None
-    h = hashlib.sha256()
-    for f in rec["sources"]:
-        h.update(open(os.path.join(ROOT, f), "rb").read())
-    if h.hexdigest() != rec["sources_sha256"]:
+    if sources_digest(rec["sources"]) != rec["sources_sha256"]:
         return None
     return rec["traffic_bytes_per_launch"]
+
+
+def sources_digest(paths) -> str:
+    """sha256 of the C++/CUDA sources with comments and whitespace removed, so
+    that editing a comment does not count as changing the kernel."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for f in paths:
+        text = open(os.path.join(ROOT, f)).read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
+    return h.hexdigest()
 
 
 def run_ours(args):

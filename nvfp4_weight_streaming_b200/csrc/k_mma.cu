@@ -5,13 +5,13 @@
 // (1 + drafted tokens checked in one pass; page "InventDB Sparkle", section
 // "How it answers quickly"). The weight read is the whole cost (page
 // "Qwen3.8-27B-NVFP4-RTX5090 API & Inference Endpoint", section "Why lm_head
-// is NVFP4, and why MTP is gone"), so the kernel is a weight stream:
+// is NVFP4, and why MTP is gone"), so the kernel is a weight stream, one CTA
+// per SM:
 //
 //   warp 0       TMA producer: 256-row x 256-element tiles of packed codes
-//                (32 KB, 128-byte swizzle) and their E4M3 scales (4 KB) into a
-//                4-stage shared-memory ring (mbarrier full/empty pairs): about
-//                144 KB in flight per SM, what the ~2.6 us loaded DRAM latency
-//                of B200 needs at full bandwidth.
+//                (32 KB, 128-byte swizzle) and their E4M3 scales (4 KB), with
+//                an L2 evict-first policy, into a ring of 3..8 shared-memory
+//                stages (mbarrier full/empty pairs).
 //   warps 1..16  consumers: warp w owns rows 16(w-1)..16(w-1)+15 of every tile.
 //                Lane (g, t) reads rows g and g+8, 64 consecutive K elements
 //                each (two swizzled 16-byte chunks and 4 scale bytes per row),
@@ -21,15 +21,20 @@
 //                the A fragment registers, then issues the MMAs. MMA i of a
 //                step maps its K slots to physical K as (2t, 2t+1) <-> 64t + 4i
 //                + {0, 1} and (2t+8, 2t+9) <-> 64t + 4i + {2, 3}, so every
-//                fragment is four consecutive elements of one lane.
+//                fragment is four consecutive elements of one lane. A warp
+//                releases a stage after its MMAs.
+//   warp 17      settler: completes tiles split between CTAs (below).
 //
-// B is X, kept for the CTA's K-slice in shared memory as f16, scaled per token
-// by a power of two (largest magnitude at 2^14) in a hi plane (exact within
-// 2^28 of that maximum) and a lo plane scaled by 2^29 (the next 29 binades);
-// elements further below are dropped. B fragments are 8-byte shared loads,
-// XOR-swizzled so a half warp touches 16 distinct bank pairs. Every product is
-// exact; only the fp32 accumulation rounds. For M > 8 the lo tiles are issued
-// only when some element of the slice needs them.
+// B is X in f16, scaled per token by a power of two (largest magnitude at
+// 2^14) in a hi plane (exact within 2^28 of that maximum) and a lo plane
+// scaled by 2^29 (the next 29 binades); elements further below are dropped.
+// Columns are groups of 64 elements padded to 136 bytes, so B fragments are
+// bank-conflict-free 8-byte shared loads at immediate offsets. Every product
+// is exact; only the fp32 accumulation rounds. When no element needs the lo
+// plane, only hi tiles are issued. M <= 4: each CTA stages its K-slice of X in
+// shared memory. M >= 5 ("X in the ring"): k_xprep writes both planes once per
+// call into the workspace and every ring stage also carries one K-step box of
+// them, so these classes need no K-slices.
 //
 // Why not tcgen05 here: on B200 a tcgen05.mma kind::f16 with M = 128 costs ~85
 // cycles whatever N <= 128 is, i.e. at most 24 weight elements per clock per
@@ -37,15 +42,16 @@
 // weight elements per clock at N = 8. For this skinny contraction the warp
 // MMA is the faster tensor path (the tcgen05 kernel is kept as variant TC).
 //
-// Work split: K is cut into S slices (an X slice fits in shared memory next
-// to the ring); the CTAs of a slice share its (256-row tile, 256-k step) units
-// evenly (stream-K). Tiles a CTA covers entirely are stored directly; a tile
-// split between CTAs writes fp32 partials, and after its last unit each CTA
-// settles its split tiles: the last piece to arrive (atomic counter per tile)
-// sums all pieces in k order, so results repeat bit for bit, and resets the
-// counter. Every mbarrier wait is bounded; on expiry the CTA records the
-// timeout in the workspace status word, stops, drains its in-flight TMA loads
-// and returns.
+// Work split: K is cut into S slices (S = 1 unless a staged X slice would not
+// fit next to the ring); the CTAs of a slice share its (256-row tile, 256-k
+// step) units evenly (stream-K). Tiles a CTA covers entirely are stored
+// directly. A split tile is completed per 16-row group: the pieces write fp32
+// partials and count themselves on the group's counter; the last sums all
+// pieces in k order (results repeat bit for bit) and resets the counter. The
+// piece at the end of a CTA's range usually finds the tile's other piece
+// already counted and finishes the tile from its registers. Every mbarrier
+// wait is bounded; on expiry the CTA records the timeout in the workspace
+// status word, stops, drains its in-flight TMA loads and returns.
 #include "kernels.h"
 #include "nvfp4_device.cuh"
 
