@@ -76,3 +76,47 @@ def test_bench_traffic_record_matches_current_kernel_sources():
     assert t is None or 100e6 < t < 120e6
     assert bench.measured_traffic("mma", "some other workload") is None
     assert bench.measured_traffic("tc", "decode projection M=1 K=5120 N=34816") is None
+
+
+def _bnd_in(lo, hi, L, W):
+    """Transcription of the kernels' closed form (unsigned 32-bit steps): the
+    number of CTA range boundaries floor(c * L / W), 1 <= c < W, in (lo, hi]."""
+    if hi <= lo:
+        return 0
+    u = 0xFFFFFFFF
+    cmin = ((((lo + 1) * W) & u) + L - 1) // L
+    cmax = ((((hi + 1) * W) & u) + L - 1) // L - 1
+    cmin = max(cmin, 1)
+    cmax = min(cmax, W - 1)
+    return cmax - cmin + 1 if cmax >= cmin else 0
+
+
+def test_piece_ordinal_closed_form_matches_enumeration():
+    """Stream-K bookkeeping: the ordinal of a piece of a split tile and the
+    number of pieces of a tile, as the kernels compute them, equal a direct
+    enumeration of the CTA ranges [c*L/W, (c+1)*L/W)."""
+    import random
+    rnd = random.Random(0)
+    cases = [(136 * 20, 148), (20 * 68, 148), (20 * 23, 49), (970 * 20, 148), (4 * 32, 128)]
+    cases += [(rnd.randint(1, 4000), rnd.randint(1, 160)) for _ in range(300)]
+    for L, W in cases:
+        if W > L:
+            W = L
+        bounds = sorted({c * L // W for c in range(1, W)})
+        for _ in range(40):
+            lo = rnd.randint(-1, L - 1)
+            hi = rnd.randint(lo, L - 1)
+            expect = sum(1 for bnd in bounds if lo < bnd <= hi)
+            assert _bnd_in(lo, hi, L, W) == expect, (L, W, lo, hi)
+        # every tile's piece count for a tile length `cnt` dividing L
+        for cnt in (c for c in (5, 20, 23, 68) if L % c == 0):
+            for t in range(L // cnt):
+                pieces = 1 + sum(1 for b in bounds if t * cnt < b <= (t + 1) * cnt - 1)
+                assert 1 + _bnd_in(t * cnt, (t + 1) * cnt - 1, L, W) == pieces
+
+
+def test_piece_arithmetic_fits_32_bits_for_the_workloads():
+    """configure() refuses plans where (units + 1) * P overflows 31 bits; the
+    benchmark shapes are far from that."""
+    for tiles, steps in ((136, 20), (20, 68), (970, 20), (136, 5)):
+        assert (tiles * (steps + 1) + 1) * 148 < 2 ** 31
