@@ -120,3 +120,27 @@ def test_piece_arithmetic_fits_32_bits_for_the_workloads():
     benchmark shapes are far from that."""
     for tiles, steps in ((136, 20), (20, 68), (970, 20), (136, 5)):
         assert (tiles * (steps + 1) + 1) * 148 < 2 ** 31
+
+
+def test_reference_arm_prints_the_contract_line():
+    """bench.py --impl reference (the oracle on the host cores) prints one JSON
+    line with the fields the contract asks of the reference arm."""
+    import json
+    import subprocess
+    import sys
+    from tests.conftest import ROOT
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                          "--warmup", "1", "--reference-rows", "256"], cwd=ROOT,
+                         capture_output=True, text=True, timeout=600, check=True).stdout
+    lines = [l for l in out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert "workload" in d["config"]
