@@ -279,7 +279,7 @@ def time_problem(pb: Problem, steps: int, warmup: int, world: int, graph_len: in
     sec = e0.elapsed_time(e1) / 1e3
     pb.check_status()
     del graph, tail_graph
-    return max_over_ranks(world, sec) / steps, steps
+    return max_over_ranks(world, sec) / steps, steps * pb.nv.nvfp4_linear_launches_per_run(pb.plan)
 
 
 def time_e2e(pb: Problem, steps: int, world: int):

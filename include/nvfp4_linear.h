@@ -110,6 +110,12 @@ size_t nvfp4_linear_workspace_bytes(nvfp4_plan_t plan);
 int nvfp4_linear_variant(nvfp4_plan_t plan);
 int nvfp4_linear_split_k(nvfp4_plan_t plan);
 
+/* Kernels one nvfp4_linear_run (or nvfp4_linear_run_static) of this plan
+ * launches: 2 for the mma variant with M >= 5 (X is converted to its two f16
+ * planes by a kernel of its own first), 1 otherwise, 0 when N == 0; -1 if the
+ * plan is null. Host-only; touches no device. */
+int nvfp4_linear_launches_per_run(nvfp4_plan_t plan);
+
 /* Run the linear on `stream` (device pointers, see the layout above):
  *   w_packed  uint8 [N][K/2]     w_scales uint8 [N][K/16] (E4M3)
  *   w_global  fp32 [1]           x        bf16 [M][K]       y bf16 [M][N]

@@ -23,7 +23,8 @@ __all__ = [
     "NVFP4_PLAN_PDL", "NVFP4_PLAN_TEST_STALL",
     "Nvfp4Error", "lib", "library_path",
     "nvfp4_linear_plan", "nvfp4_linear_workspace_bytes", "nvfp4_linear_variant",
-    "nvfp4_linear_split_k", "nvfp4_linear_run", "nvfp4_linear_run_static",
+    "nvfp4_linear_split_k", "nvfp4_linear_launches_per_run", "nvfp4_linear_run",
+    "nvfp4_linear_run_static",
     "NVFP4_STATIC_SCRATCH_BYTES", "nvfp4_linear_status", "nvfp4_linear_destroy",
     "nvfp4_pack_check", "nvfp4_quantize", "nvfp4_status_string", "EXPORTS",
 ]
@@ -54,6 +55,7 @@ EXPORTS = {
     "nvfp4_linear_workspace_bytes": (_c.c_size_t, [_P]),
     "nvfp4_linear_variant": (_c.c_int, [_P]),
     "nvfp4_linear_split_k": (_c.c_int, [_P]),
+    "nvfp4_linear_launches_per_run": (_c.c_int, [_P]),
     "nvfp4_linear_run": (_c.c_int, [_P, _P, _P, _P, _P, _P, _P, _c.c_size_t, _P]),
     "nvfp4_linear_run_static": (_c.c_int, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "nvfp4_linear_status": (_c.c_int, [_P, _P, _P]),
@@ -141,6 +143,10 @@ def nvfp4_linear_variant(plan) -> int:
 
 def nvfp4_linear_split_k(plan) -> int:
     return int(lib().nvfp4_linear_split_k(plan))
+
+
+def nvfp4_linear_launches_per_run(plan) -> int:
+    return int(lib().nvfp4_linear_launches_per_run(plan))
 
 
 def nvfp4_linear_run(plan, w_packed, w_scales, w_global, x, y, workspace=None, ws_bytes=None,

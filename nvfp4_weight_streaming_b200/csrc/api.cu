@@ -208,6 +208,12 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
 size_t nvfp4_linear_workspace_bytes(nvfp4_plan_t plan) { return plan ? plan->ws_bytes : 0; }
 int nvfp4_linear_variant(nvfp4_plan_t plan) { return plan ? plan->variant : -1; }
 int nvfp4_linear_split_k(nvfp4_plan_t plan) { return plan ? plan->split_k : -1; }
+int nvfp4_linear_launches_per_run(nvfp4_plan_t plan) {
+  if (!plan) return -1;
+  if (plan->N == 0) return 0;
+  if (plan->K > 0 && plan->variant == NVFP4_VARIANT_MMA && plan->mma.xr) return 2;
+  return 1;
+}
 
 void nvfp4_linear_destroy(nvfp4_plan_t plan) { delete plan; }
 

@@ -53,6 +53,7 @@ def test_null_arguments_rejected():
     assert L.nvfp4_linear_status(None, None, None) == nv.NVFP4_ERR_INVALID_ARG
     assert L.nvfp4_linear_workspace_bytes(None) == 0
     assert L.nvfp4_linear_variant(None) == -1
+    assert L.nvfp4_linear_launches_per_run(None) == -1
     L.nvfp4_linear_destroy(None)
     assert L.nvfp4_pack_check(None, None, None, 4, 17, None, None, None) == \
         nv.NVFP4_ERR_INVALID_ARG

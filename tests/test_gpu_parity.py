@@ -327,6 +327,22 @@ def test_linear_k_zero_writes_zeros_and_n_zero_is_noop():
     nv.nvfp4_linear_destroy(plan)
 
 
+def test_launches_per_run_counts_the_x_conversion_kernel():
+    """The mma variant with M >= 5 converts X in a kernel of its own before
+    the main kernel; every other plan launches one kernel, N == 0 none."""
+    d = torch.cuda.current_device()
+    cases = [(nv.NVFP4_VARIANT_MMA, 1, 1024, 5120, 1), (nv.NVFP4_VARIANT_MMA, 4, 1024, 5120, 1),
+             (nv.NVFP4_VARIANT_MMA, 5, 1024, 5120, 2), (nv.NVFP4_VARIANT_MMA, 16, 1024, 5120, 2),
+             (nv.NVFP4_VARIANT_TC, 16, 1024, 5120, 1), (nv.NVFP4_VARIANT_GEMV, 1, 1024, 5120, 1),
+             (nv.NVFP4_VARIANT_MMA, 8, 1024, 0, 1), (nv.NVFP4_VARIANT_AUTO, 1, 0, 256, 0)]
+    for variant, M, N, K, want in cases:
+        plan = nv.nvfp4_linear_plan(M, N, K, d, variant)
+        try:
+            assert nv.nvfp4_linear_launches_per_run(plan) == want, (variant, M, N, K)
+        finally:
+            nv.nvfp4_linear_destroy(plan)
+
+
 @pytest.mark.parametrize("variant", [nv.NVFP4_VARIANT_TC, nv.NVFP4_VARIANT_MMA])
 def test_forced_timeout_reports_status_and_recovers(variant):
     """Test-only flag: the TMA producer never signals, every bounded wait runs
