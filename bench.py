@@ -487,7 +487,9 @@ def run_reference(args):
     sample = ("each step: fp64 oracle linear on the first %d of %d rows of the %s workload "
               "(M=%d, K=%d), bytes scaled to the sample" % (rows, wl.N, args.workload, M, wl.K))
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": 1,
+        # n_gpus is the launch's world size; the oracle itself runs on rank 0's host cores only
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
