@@ -42,9 +42,10 @@
  *   - Limits: 1 <= M <= 16, N >= 0, K >= 0 with K % 256 == 0, every pointer
  *     16-byte aligned (gs: 4-byte aligned). N need not be a multiple of any
  *     tile size.
- *   - Thread safety: plans are immutable after creation and may be shared by
- *     threads; runs on different streams may proceed concurrently if they use
- *     different workspaces.
+ *   - Thread safety: a plan's launch parameters are fixed at creation; the
+ *     TMA descriptors it caches per buffer are updated under a lock, so a
+ *     plan may be shared by threads. Runs on different streams may proceed
+ *     concurrently if they use different workspaces.
  */
 #ifndef NVFP4_LINEAR_H
 #define NVFP4_LINEAR_H
@@ -69,8 +70,8 @@ typedef enum {
 
 typedef struct nvfp4_plan_s* nvfp4_plan_t;
 
-/* Kernel variants (plan flags, bits 0..3). AUTO picks per (M, N, K) from a
- * table of bandwidths measured on B200. */
+/* Kernel variants (plan flags, bits 0..3). AUTO takes MMA, the fastest on
+ * B200 for every M measured, and TC for a shape MMA cannot take. */
 #define NVFP4_VARIANT_AUTO 0u
 #define NVFP4_VARIANT_GEMV 1u  /* CUDA-core warp-per-row GEMV, fp32 FMA        */
 #define NVFP4_VARIANT_MMA  2u  /* TMA ring + warp MMA (m16n8k16), stream-K    */
