@@ -12,6 +12,10 @@ Every function cites, in the C++ source, the passage it follows:
     4-bit codes are stored packed in uint8 tensors.
   * "InventDB Sparkle", section "How it answers quickly": the weight read per
     token and the one-pass check of drafted tokens (M = 1..16).
+  * "SparkInfer" README, sections "Layout & scoring" (fused FFN kernels) and
+    "DSpark speculative decode" (greedy decoding); "Qwen3.8-27B-NVFP4-RTX5090
+    API & Inference Endpoint", section "SparkInfer + DSpark" (near ties at the
+    top of the logits): the SwiGLU and argmax / top-k epilogues.
 """
 from __future__ import annotations
 
@@ -67,6 +71,10 @@ def _load():
             "ora_count_bad": (c.c_int64, [P, c.c_int64, c.c_float]),
             "ora_linear": (c.c_int, [P, P, c.c_float, P, c.c_int64, c.c_int64, c.c_int64,
                                      P, c.c_int64, P, P, c.c_int]),
+            "ora_silu": (c.c_double, [c.c_double]),
+            "ora_swiglu_linear": (c.c_int, [P, P, c.c_float, P, c.c_int64, c.c_int64, c.c_int64,
+                                            P, c.c_int64, P, P, P, P, P, c.c_int]),
+            "ora_topk": (c.c_int, [P, c.c_int64, c.c_int64, c.c_int64, P]),
             "ora_bf16_rne": (c.c_uint16, [c.c_double]),
             "ora_bf16_value": (c.c_double, [c.c_uint16]),
             "ora_bytes_model": (c.c_double, [c.c_int64, c.c_int64, c.c_int64]),
@@ -205,6 +213,76 @@ def linear(packed, scales, gs, x_bf16, M, N, K, rows=None, nthreads: int = NTHRE
 def tolerance(y_ref: np.ndarray, absdot: np.ndarray) -> np.ndarray:
     """Per-element bound |y - y_ref| <= 1e-2 |y_ref| + 1e-4 sum_k |w_hat x|."""
     return 1e-2 * np.abs(y_ref) + 1e-4 * absdot
+
+
+def silu(v: float) -> float:
+    return float(_load().ora_silu(float(v)))
+
+
+def swiglu_linear(packed, scales, gs, x_bf16, M, N2, K, cols=None, nthreads: int = NTHREADS):
+    """SiLU-gated output of a fused gate+up projection (rows 2c, 2c+1 = gate,
+    up of output column c). Returns (h, gate, up, absdot_gate, absdot_up),
+    each fp64 [M][ncols]."""
+    packed = _c(packed, np.uint8)
+    scales = _c(scales, np.uint8)
+    x_bf16 = _c(x_bf16, np.uint16)
+    if cols is None:
+        ncols = N2 // 2
+        cols_arr = None
+    else:
+        cols_arr = _c(cols, np.int64)
+        ncols = cols_arr.size
+    out = [np.zeros((M, ncols), np.float64) for _ in range(5)]
+    rc = _load().ora_swiglu_linear(_ptr(packed), _ptr(scales), float(gs), _ptr(x_bf16), M, N2,
+                                   K, _ptr(cols_arr), ncols, *[_ptr(o) for o in out], nthreads)
+    if rc:
+        raise ValueError("ora_swiglu_linear failed (%d)" % rc)
+    return tuple(out)
+
+
+# sup over v of |d silu / dv| is 1.0998 (at v = 2.3994); rounded up
+SILU_LIPSCHITZ = 1.1
+
+
+def swiglu_tolerance(h_ref, gate, up, absdot_gate, absdot_up) -> np.ndarray:
+    """Bound on |h - h_ref| for a kernel whose gate and up values each meet the
+    linear's bound and whose output is rounded to bf16: with tg, tu the linear
+    bounds of gate and up and L the Lipschitz constant of SiLU,
+        |silu(g') u' - silu(g) u| <= L tg (|u| + tu) + |silu(g)| tu,
+    plus the bf16 rounding of the result (relative 2^-9, taken as 2^-8)."""
+    tg = tolerance(gate, absdot_gate)
+    tu = tolerance(up, absdot_up)
+    sg = np.abs(np.vectorize(silu, otypes=[np.float64])(gate)) if np.size(gate) else np.abs(gate)
+    b = SILU_LIPSCHITZ * tg * (np.abs(up) + tu) + sg * tu
+    return (1.0 + 2.0 ** -8) * b + 2.0 ** -8 * np.abs(h_ref)
+
+
+def topk(y, k: int) -> np.ndarray:
+    """Indices [M][k] of the k largest entries of each row of y (fp64 [M][N]),
+    largest first, ties by ascending index; k = 1 is the greedy argmax."""
+    y = _c(np.atleast_2d(y), np.float64)
+    M, N = y.shape
+    idx = np.zeros((M, k), np.int64)
+    rc = _load().ora_topk(_ptr(y), M, N, k, _ptr(idx))
+    if rc:
+        raise ValueError("ora_topk failed (%d)" % rc)
+    return idx
+
+
+def argmax_decided(y_ref, tol) -> tuple:
+    """(argmax [M], decided [M]): the oracle's greedy choice per row, and
+    whether it is decided within tolerance, i.e. the reference top-2 gap
+    exceeds the sum of the two logits' bounds (else a kernel may pick the
+    runner-up; reading R10)."""
+    y_ref = np.atleast_2d(np.asarray(y_ref, np.float64))
+    tol = np.atleast_2d(np.asarray(tol, np.float64))
+    if y_ref.shape[1] < 2:
+        return topk(y_ref, 1)[:, 0], np.ones(y_ref.shape[0], bool)
+    t2 = topk(y_ref, 2)
+    r = np.arange(y_ref.shape[0])
+    a, b = t2[:, 0], t2[:, 1]
+    decided = y_ref[r, a] - y_ref[r, b] > tol[r, a] + tol[r, b]
+    return a, decided
 
 
 def bf16_round_array(v: np.ndarray) -> np.ndarray:

@@ -271,6 +271,69 @@ int ora_linear(const uint8_t* packed, const uint8_t* scales, float gs,
   return 0;
 }
 
+// SiLU(v) = v * sigmoid(v) = v / (1 + e^-v). For v below about -709, e^-v
+// overflows to +inf and the quotient is -0.0, the limit of SiLU there.
+double ora_silu(double v) { return v / (1.0 + std::exp(-v)); }
+
+// Gated output of a fused gate+up projection (reading R11): weight rows 2c
+// and 2c+1 are the gate and up rows of output column c. Both dot products are
+// taken by ora_linear (same exact dequantisation, fp64 sums); the gate passes
+// through SiLU and multiplies the up value, all in fp64.
+int ora_swiglu_linear(const uint8_t* packed, const uint8_t* scales, float gs,
+                      const uint16_t* x_bf16, int64_t M, int64_t N2, int64_t K,
+                      const int64_t* cols, int64_t ncols, double* h, double* gate,
+                      double* up, double* absdot_gate, double* absdot_up, int nthreads) {
+  if (M < 0 || N2 < 0 || N2 % 2 != 0 || ncols < 0) return -1;
+  if (!cols && ncols != N2 / 2) return -1;
+  if (ncols == 0 || M == 0) return 0;
+  if (!h) return -1;
+  std::vector<int64_t> rows(size_t(2 * ncols));
+  for (int64_t c = 0; c < ncols; ++c) {
+    int64_t col = cols ? cols[c] : c;
+    if (col < 0 || col >= N2 / 2) return -1;
+    rows[size_t(c)] = 2 * col;                 // gate rows first ...
+    rows[size_t(ncols + c)] = 2 * col + 1;     // ... then the matching up rows
+  }
+  std::vector<double> y(size_t(M * 2 * ncols)), ad(size_t(M * 2 * ncols));
+  int st = ora_linear(packed, scales, gs, x_bf16, M, N2, K, rows.data(), 2 * ncols,
+                      y.data(), ad.data(), nthreads);
+  if (st != 0) return st;
+  for (int64_t m = 0; m < M; ++m) {
+    for (int64_t c = 0; c < ncols; ++c) {
+      double g = y[size_t(m * 2 * ncols + c)];
+      double u = y[size_t(m * 2 * ncols + ncols + c)];
+      h[m * ncols + c] = ora_silu(g) * u;
+      if (gate) gate[m * ncols + c] = g;
+      if (up) up[m * ncols + c] = u;
+      if (absdot_gate) absdot_gate[m * ncols + c] = ad[size_t(m * 2 * ncols + c)];
+      if (absdot_up) absdot_up[m * ncols + c] = ad[size_t(m * 2 * ncols + ncols + c)];
+    }
+  }
+  return 0;
+}
+
+// The k largest entries of each row of y [M][N], largest first; equal values
+// are ordered by ascending index (reading R10: the lowest index wins a tie).
+// k = 1 is the greedy argmax.
+int ora_topk(const double* y, int64_t M, int64_t N, int64_t k, int64_t* idx) {
+  if (M < 0 || N < 0 || k < 0 || k > N) return -1;
+  if (M == 0 || k == 0) return 0;
+  if (!y || !idx) return -1;
+  for (int64_t i = 0; i < M * N; ++i)
+    if (std::isnan(y[i])) return -3;
+  std::vector<int64_t> order(static_cast<size_t>(N));
+  for (int64_t m = 0; m < M; ++m) {
+    const double* row = y + m * N;
+    for (int64_t j = 0; j < N; ++j) order[size_t(j)] = j;
+    auto before = [row](int64_t a, int64_t b) {
+      return row[a] > row[b] || (row[a] == row[b] && a < b);
+    };
+    std::partial_sort(order.begin(), order.begin() + k, order.end(), before);
+    for (int64_t j = 0; j < k; ++j) idx[m * k + j] = order[size_t(j)];
+  }
+  return 0;
+}
+
 double ora_bytes_model(int64_t M, int64_t N, int64_t K) {
   return double(N) * double(K) / 2.0 + double(N) * double(K) / 16.0 +
          2.0 * double(M) * double(K) + 2.0 * double(M) * double(N);

@@ -18,6 +18,15 @@
  *     Inference Endpoint", section "Recipe (NVIDIA ModelOpt)": weights are
  *     NVFP4 with 16-element scale groups; section "Serving": the checkpoint
  *     keeps the 4-bit codes packed two to a byte (uint8 tensors).
+ *   - Two epilogues of that linear: the SiLU-gated output of a fused gate+up
+ *     projection (page "SparkInfer" README, section "Layout & scoring": the
+ *     engine's FFN kernels are fused; page "Qwen3.8-27B-NVFP4-RTX5090 API &
+ *     Inference Endpoint", section "Recipe (NVIDIA ModelOpt)": the MLP is
+ *     NVFP4), and the greedy argmax / top-k of the logits (page "SparkInfer"
+ *     README, section "DSpark speculative decode": greedy decoding; page
+ *     "Qwen3.8-27B-NVFP4-RTX5090 API & Inference Endpoint", section
+ *     "SparkInfer + DSpark": a verify pass keeps a drafted token only where it
+ *     equals the target's own choice, and near ties at the top can flip).
  *   - The reference linear Y[M,N] = X[M,K] * W^T with W dequantised exactly and
  *     the sum accumulated in fp64. Page "InventDB Sparkle", section "How it
  *     answers quickly" (decode reads every weight once per token; the
@@ -34,6 +43,10 @@
  *   R6 values that round to zero get code 0x0, never 0x8.
  *   R7 every quantiser step is an fp32 operation in the order written in
  *      ora_quantize (the decisions are taken on fp32 values).
+ *   R10 an argmax or top-k tie goes to the lowest index.
+ *   R11 a fused gate+up projection interleaves its rows: row 2c is the gate
+ *      and row 2c+1 the up row of output column c; the gated output is
+ *      silu(gate) * up (the SiLU-gated MLP of the model family).
  *
  * Parity pins: every function here is pinned by tests under tests/ that do not
  * call back into the same code path (exhaustive tables, brute force, closed
@@ -97,6 +110,27 @@ int ora_linear(const uint8_t* packed, const uint8_t* scales, float gs,
                const uint16_t* x_bf16, int64_t M, int64_t N, int64_t K,
                const int64_t* rows, int64_t nrows, double* y, double* absdot,
                int nthreads);
+
+/* SiLU(v) = v * sigmoid(v) = v / (1 + exp(-v)), fp64. */
+double ora_silu(double v);
+
+/* Gated (SwiGLU) output of a fused gate+up projection W [N2][K], N2 even.
+ * Reading R11: rows 2c and 2c+1 of W are the gate and up rows of output column
+ * c. For the columns listed in cols[0..ncols) (NULL means 0..N2/2-1 and ncols
+ * must equal N2/2):
+ *   gate[m][i] = sum_k w_hat[2c][k] x[m][k],  up[m][i] = sum_k w_hat[2c+1][k] x[m][k]
+ *   h[m][i]    = silu(gate[m][i]) * up[m][i]            (all fp64, c = cols[i])
+ * gate, up and the absdot sums of each (for the tolerance bound) are nullable
+ * outputs, each [M][ncols]. Returns 0, or -1 on bad arguments. */
+int ora_swiglu_linear(const uint8_t* packed, const uint8_t* scales, float gs,
+                      const uint16_t* x_bf16, int64_t M, int64_t N2, int64_t K,
+                      const int64_t* cols, int64_t ncols, double* h, double* gate,
+                      double* up, double* absdot_gate, double* absdot_up, int nthreads);
+
+/* Indices of the k largest entries of each row of y [M][N], largest first,
+ * equal values by ascending index (reading R10); idx is [M][k]. k = 1 is the
+ * greedy argmax. Returns 0, -1 on bad arguments, -3 if y holds a NaN. */
+int ora_topk(const double* y, int64_t M, int64_t N, int64_t k, int64_t* idx);
 
 /* Round an fp64 value to bf16 (round to nearest even, overflow to inf), as bits. */
 uint16_t ora_bf16_rne(double v);

@@ -36,6 +36,17 @@ MUTANTS = {
     "X indexed transposed": (
         "double p = wrow[size_t(k)] * xm[k];",
         "double p = wrow[size_t(k)] * x[size_t(k * M + m) % size_t(M * K)];"),
+    "SiLU gate sign flipped": (
+        "return v / (1.0 + std::exp(-v));",
+        "return v / (1.0 + std::exp(v));"),
+    "gate and up rows swapped": (
+        "rows[size_t(c)] = 2 * col;                 // gate rows first ...\n"
+        "    rows[size_t(ncols + c)] = 2 * col + 1;",
+        "rows[size_t(c)] = 2 * col + 1;\n"
+        "    rows[size_t(ncols + c)] = 2 * col;"),
+    "top-k ties to the highest index": (
+        "(row[a] == row[b] && a < b)",
+        "(row[a] == row[b] && a > b)"),
     "last product of each row dropped": (
         "for (int64_t k = 0; k < K; ++k) {\n          double p",
         "for (int64_t k = 0; k < K - 1; ++k) {\n          double p"),

@@ -371,3 +371,129 @@ def test_bytes_model_matches_pages_lm_head():
     assert round(N * K * 2 / 1e9, 2) == d["bf16_gb"]
     # X and Y terms: 2*M*K + 2*M*N
     assert oracle.bytes_model(16, N, K) - nvfp4 == 2 * 16 * K + 2 * 16 * N
+
+
+# ----- epilogues: SwiGLU and greedy argmax / top-k ---------------------------
+
+def _silu_expit(v):
+    """SiLU from SciPy's logistic function (independent library code)."""
+    from scipy.special import expit
+    return np.asarray(v, np.float64) * expit(np.asarray(v, np.float64))
+
+
+def test_silu_closed_forms():
+    assert oracle.silu(0.0) == 0.0
+    # sigmoid(ln r) = r / (1 + r) exactly, so silu(ln r) = ln(r) r / (1 + r)
+    for r in (0.125, 0.5, 2.0, 3.0, 7.0, 1000.0):
+        v = math.log(r)
+        assert oracle.silu(v) == pytest.approx(v * r / (1.0 + r), rel=1e-15)
+    # odd part: silu(v) - silu(-v) = v
+    for v in np.linspace(-30.0, 30.0, 241):
+        assert oracle.silu(v) - oracle.silu(-v) == pytest.approx(v, rel=1e-14, abs=1e-300)
+    # tails: the limits v and 0
+    assert oracle.silu(800.0) == 800.0 and oracle.silu(40.0) == pytest.approx(40.0, rel=1e-16)
+    assert oracle.silu(-800.0) == 0.0
+    rng = np.random.default_rng(3)
+    for v in rng.normal(0.0, 6.0, 200):
+        assert oracle.silu(v) == pytest.approx(float(_silu_expit(v)), rel=1e-13, abs=1e-300)
+
+
+def test_swiglu_pairs_rows_and_gates_with_silu():
+    """Against an independent construction: torch/grid decode of W, numpy
+    matmul of the even (gate) and odd (up) rows, SciPy's logistic."""
+    wl = synth.WORKLOADS["tiny"]
+    p, s, gs = oracle.quantize(synth.weights_f32(wl))
+    M = 3
+    X = synth.x_bf16_custom(synth.X_NORMAL, M, wl.K, seed=4)
+    x = oracle.bf16_bits_to_f64(X)
+    W = independent_dequant(p, s, gs, wl.N, wl.K)
+    g_ref, u_ref = x @ W[0::2].T, x @ W[1::2].T
+    h, g, u, adg, adu = oracle.swiglu_linear(p, s, gs, X, M, wl.N, wl.K)
+    assert h.shape == (M, wl.N // 2)
+    assert np.allclose(g, g_ref, rtol=1e-12, atol=1e-15)
+    assert np.allclose(u, u_ref, rtol=1e-12, atol=1e-15)
+    assert np.allclose(h, _silu_expit(g_ref) * u_ref, rtol=1e-11, atol=1e-15)
+    assert np.allclose(adg, np.abs(x) @ np.abs(W[0::2]).T, rtol=1e-12)
+    assert np.allclose(adu, np.abs(x) @ np.abs(W[1::2]).T, rtol=1e-12)
+    cols = np.array([255, 0, 7, 7])
+    hc, gc, uc, _, _ = oracle.swiglu_linear(p, s, gs, X, M, wl.N, wl.K, cols=cols)
+    assert np.array_equal(hc, h[:, cols]) and np.array_equal(gc, g[:, cols])
+    assert np.array_equal(uc, u[:, cols])
+
+
+def test_swiglu_one_hot_exact_values():
+    """gs = 1 and X = e_k: gate and up are single decoded weights, and at
+    0, +-2688 (= 6 * 448) SiLU is exact in fp64, so h is known exactly."""
+    K = 16
+    # columns: (gate code, gate scale, up code, up scale) -> h
+    table = [(0x0, 0x38, 0x2, 0x38, 0.0),             # gate 0
+             (0x7, 0x7E, 0x3, 0x38, 2688.0 * 1.5),    # gate 2688, up 1.5
+             (0xF, 0x7E, 0x7, 0x40, -0.0),            # gate -2688: silu = -0
+             (0x7, 0x7E, 0x0, 0x38, 0.0)]             # up 0
+    N2 = 2 * len(table)
+    codes = np.zeros((N2, K), np.uint8)
+    sc = np.zeros((N2, 1), np.uint8)
+    for c, (gc, gsc, uc, usc, _) in enumerate(table):
+        codes[2 * c, :] = gc
+        sc[2 * c] = gsc
+        codes[2 * c + 1, :] = uc
+        sc[2 * c + 1] = usc
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    for k in (0, 5, 15):
+        X = np.zeros((1, K), np.uint16)
+        X[0, k] = 0x3F80
+        h, g, u, _, _ = oracle.swiglu_linear(packed, sc, 1.0, X, 1, N2, K)
+        assert [abs(v) for v in h[0]] == [abs(t[4]) for t in table]
+        assert g[0, 1] == 2688.0 and g[0, 2] == -2688.0 and u[0, 1] == 1.5
+
+
+def test_swiglu_tolerance_covers_perturbed_gate_and_up():
+    """The derived bound holds for gate and up values perturbed anywhere
+    within their own linear bounds, the result rounded to bf16 (torch)."""
+    assert oracle.SILU_LIPSCHITZ >= 1.0998
+    v = np.linspace(-20.0, 20.0, 400001)
+    slope = np.abs(np.diff(_silu_expit(v)) / np.diff(v))
+    assert slope.max() <= oracle.SILU_LIPSCHITZ and slope.max() > 1.09
+    rng = np.random.default_rng(5)
+    n = 4000
+    g = rng.uniform(-12.0, 12.0, n)
+    u = rng.uniform(-5.0, 5.0, n)
+    adg = np.abs(g) * rng.uniform(1.0, 40.0, n)
+    adu = np.abs(u) * rng.uniform(1.0, 40.0, n)
+    h_ref = _silu_expit(g) * u
+    bound = oracle.swiglu_tolerance(h_ref, g, u, adg, adu)
+    tg, tu = oracle.tolerance(g, adg), oracle.tolerance(u, adu)
+    for sg, su in ((1, 1), (1, -1), (-1, 1), (-1, -1), (None, None)):
+        if sg is None:
+            dg, du = rng.uniform(-1, 1, n) * tg, rng.uniform(-1, 1, n) * tu
+        else:
+            dg, du = sg * tg, su * tu
+        h = _silu_expit(g + dg) * (u + du)
+        hb = torch.tensor(h).to(torch.bfloat16).to(torch.float64).numpy()
+        assert np.all(np.abs(hb - h_ref) <= bound)
+
+
+def test_topk_matches_sorting_bruteforce():
+    rng = np.random.default_rng(7)
+    y = rng.integers(0, 5, size=(6, 13)).astype(np.float64)   # many ties
+    y[5] = 2.0                                                # all equal
+    for k in range(1, 14):
+        got = oracle.topk(y, k)
+        for m in range(y.shape[0]):
+            want = sorted(range(y.shape[1]), key=lambda j: (-y[m, j], j))[:k]
+            assert list(got[m]) == want, (m, k)
+    assert np.array_equal(oracle.topk(y, 1)[:, 0], np.argmax(y, axis=1))  # first maximum
+    z = rng.normal(size=(4, 1000))
+    assert np.array_equal(oracle.topk(z, 20), np.argsort(-z, axis=1, kind="stable")[:, :20])
+    with pytest.raises(ValueError):
+        oracle.topk(np.array([[1.0, float("nan")]]), 1)
+
+
+def test_argmax_decided_uses_both_bounds():
+    y = np.array([[1.0, 0.9, 0.0], [1.0, 0.99, 0.0], [0.5, 0.5, 0.1], [0.0, 3.0, 2.0]])
+    tol = np.full_like(y, 0.01)
+    idx, dec = oracle.argmax_decided(y, tol)
+    assert list(idx) == [0, 0, 0, 1]
+    assert list(dec) == [True, False, False, True]
+    idx1, dec1 = oracle.argmax_decided(np.array([[4.0]]), np.array([[1.0]]))
+    assert list(idx1) == [0] and list(dec1) == [True]
