@@ -16,6 +16,10 @@ Every function cites, in the C++ source, the passage it follows:
     "DSpark speculative decode" (greedy decoding); "Qwen3.8-27B-NVFP4-RTX5090
     API & Inference Endpoint", section "SparkInfer + DSpark" (near ties at the
     top of the logits): the SwiGLU and argmax / top-k epilogues.
+  * "Qwen3.8-27B-NVFP4-RTX5090 API & Inference Endpoint", section "Recipe
+    (NVIDIA ModelOpt)" (W4A4, group size 16, per-layer input scale) and
+    "InventDB Sparkle", section "How it answers quickly" (8-bit weights): the
+    W4A4 and FP8 weight tiers.
 """
 from __future__ import annotations
 
@@ -75,6 +79,11 @@ def _load():
             "ora_swiglu_linear": (c.c_int, [P, P, c.c_float, P, c.c_int64, c.c_int64, c.c_int64,
                                             P, c.c_int64, P, P, P, P, P, c.c_int]),
             "ora_topk": (c.c_int, [P, c.c_int64, c.c_int64, c.c_int64, P]),
+            "ora_linear_w4a4": (c.c_int, [P, P, c.c_float, P, P, c.c_float, c.c_int64, c.c_int64,
+                                          c.c_int64, P, c.c_int64, P, P, c.c_int]),
+            "ora_quantize_fp8_rows": (c.c_int, [P, c.c_int64, c.c_int64, P, P, c.c_int]),
+            "ora_linear_fp8": (c.c_int, [P, P, P, c.c_int64, c.c_int64, c.c_int64, P, c.c_int64,
+                                         P, P, c.c_int]),
             "ora_bf16_rne": (c.c_uint16, [c.c_double]),
             "ora_bf16_value": (c.c_double, [c.c_uint16]),
             "ora_bytes_model": (c.c_double, [c.c_int64, c.c_int64, c.c_int64]),
@@ -283,6 +292,67 @@ def argmax_decided(y_ref, tol) -> tuple:
     a, b = t2[:, 0], t2[:, 1]
     decided = y_ref[r, a] - y_ref[r, b] > tol[r, a] + tol[r, b]
     return a, decided
+
+
+def quantize_x(x_bf16, gs_x=None, nthreads: int = NTHREADS):
+    """NVFP4 activations for the W4A4 tier: X bf16 [M][K] -> (packed [M][K/2],
+    scales [M][K/16], gs_x). gs_x is the per-tensor input scale; None takes
+    amax(|X|) / (6 * 448) of this X. The steps are the weight quantiser's."""
+    x_bf16 = _c(x_bf16, np.uint16)
+    x = bf16_bits_to_f64(x_bf16).astype(np.float32)          # exact
+    if gs_x is None:
+        gs_x = global_scale(x, nthreads)
+    packed, scales = quantize_rows(x, float(gs_x), nthreads)
+    return packed, scales, float(gs_x)
+
+
+def _rows_arg(rows, N):
+    if rows is None:
+        return None, N
+    r = _c(rows, np.int64)
+    return r, r.size
+
+
+def linear_w4a4(w_packed, w_scales, gs_w, x_packed, x_scales, gs_x, M, N, K, rows=None,
+                nthreads: int = NTHREADS):
+    """W4A4 reference linear. Returns (y fp64 [M][nrows], absdot fp64 [M][nrows])."""
+    arrs = [_c(a, np.uint8) for a in (w_packed, w_scales, x_packed, x_scales)]
+    rows_arr, nrows = _rows_arg(rows, N)
+    y = np.zeros((M, nrows), np.float64)
+    ad = np.zeros((M, nrows), np.float64)
+    rc = _load().ora_linear_w4a4(_ptr(arrs[0]), _ptr(arrs[1]), float(gs_w), _ptr(arrs[2]),
+                                 _ptr(arrs[3]), float(gs_x), M, N, K, _ptr(rows_arr), nrows,
+                                 _ptr(y), _ptr(ad), nthreads)
+    if rc:
+        raise ValueError("ora_linear_w4a4 failed (%d)" % rc)
+    return y, ad
+
+
+def quantize_fp8_rows(w, nthreads: int = NTHREADS):
+    """FP8 weight tier: w fp32 [N][K] -> (codes uint8 [N][K], row scales fp32 [N])."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    codes = np.zeros((N, K), np.uint8)
+    sc = np.zeros(N, np.float32)
+    rc = _load().ora_quantize_fp8_rows(_ptr(w), N, K, _ptr(codes), _ptr(sc), nthreads)
+    if rc:
+        raise ValueError("ora_quantize_fp8_rows failed (%d)" % rc)
+    return codes, sc
+
+
+def linear_fp8(codes, row_scales, x_bf16, M, N, K, rows=None, nthreads: int = NTHREADS):
+    """FP8 weight tier reference linear. Returns (y, absdot), fp64 [M][nrows]."""
+    codes = _c(codes, np.uint8)
+    row_scales = _c(row_scales, np.float32)
+    x_bf16 = _c(x_bf16, np.uint16)
+    rows_arr, nrows = _rows_arg(rows, N)
+    y = np.zeros((M, nrows), np.float64)
+    ad = np.zeros((M, nrows), np.float64)
+    rc = _load().ora_linear_fp8(_ptr(codes), _ptr(row_scales), _ptr(x_bf16), M, N, K,
+                                _ptr(rows_arr), nrows, _ptr(y), _ptr(ad), nthreads)
+    if rc:
+        raise ValueError("ora_linear_fp8 failed (%d)" % rc)
+    return y, ad
 
 
 def bf16_round_array(v: np.ndarray) -> np.ndarray:

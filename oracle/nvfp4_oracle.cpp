@@ -334,6 +334,100 @@ int ora_topk(const double* y, int64_t M, int64_t N, int64_t k, int64_t* idx) {
   return 0;
 }
 
+// W4A4 reference (reading R14): both operands NVFP4. X [M][K] is given as
+// codes, block scales and its own per-tensor scale, like W; each is
+// dequantised exactly by ora_dequant_f64 and the products are summed in fp64.
+int ora_linear_w4a4(const uint8_t* w_packed, const uint8_t* w_scales, float gs_w,
+                    const uint8_t* x_packed, const uint8_t* x_scales, float gs_x,
+                    int64_t M, int64_t N, int64_t K, const int64_t* rows, int64_t nrows,
+                    double* y, double* absdot, int nthreads) {
+  if (M < 0 || N < 0 || K < 0 || K % 16 != 0 || nrows < 0) return -1;
+  if (!rows && nrows != N) return -1;
+  if (nrows == 0 || M == 0) return 0;
+  if (!y || (K > 0 && (!w_packed || !w_scales || !x_packed || !x_scales))) return -1;
+  if (rows)
+    for (int64_t i = 0; i < nrows; ++i)
+      if (rows[i] < 0 || rows[i] >= N) return -1;
+  std::vector<double> xhat(size_t(M * K));
+  if (K > 0) ora_dequant_f64(x_packed, x_scales, gs_x, M, K, xhat.data());
+  split_range(nrows, nthreads, [&](int64_t lo, int64_t hi) {
+    std::vector<double> what(static_cast<size_t>(K));
+    for (int64_t i = lo; i < hi; ++i) {
+      const int64_t n = rows ? rows[i] : i;
+      if (K > 0) ora_dequant_f64(w_packed + n * (K / 2), w_scales + n * (K / 16), gs_w, 1, K,
+                                 what.data());
+      for (int64_t m = 0; m < M; ++m) {
+        double sum = 0.0, asum = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+          const double prod = what[size_t(k)] * xhat[size_t(m * K + k)];
+          sum += prod;
+          asum += std::fabs(prod);
+        }
+        y[m * nrows + i] = sum;
+        if (absdot) absdot[m * nrows + i] = asum;
+      }
+    }
+  });
+  return 0;
+}
+
+// FP8 weight tier (reading R15): one fp32 scale per output row,
+// s_n = amax(|W[n]|) / 448, and codes E4M3(w / s_n) (RNE, saturating, each
+// step one fp32 operation); a row with s_n = 0 gets all-zero codes.
+int ora_quantize_fp8_rows(const float* w, int64_t N, int64_t K, uint8_t* codes,
+                          float* row_scales, int nthreads) {
+  if (N < 0 || K < 0) return -1;
+  if (N == 0) return 0;
+  if (!w || !row_scales || (K > 0 && !codes)) return -1;
+  for (int64_t i = 0; i < N * K; ++i)
+    if (!std::isfinite(w[i])) return -2;
+  split_range(N, nthreads, [&](int64_t lo, int64_t hi) {
+    for (int64_t n = lo; n < hi; ++n) {
+      const float* row = w + n * K;
+      float amax = 0.0f;
+      for (int64_t k = 0; k < K; ++k) amax = std::max(amax, std::fabs(row[k]));
+      const float sn = amax / 448.0f;
+      row_scales[n] = sn;
+      for (int64_t k = 0; k < K; ++k)
+        codes[n * K + k] = (sn > 0.0f) ? uint8_t(ora_e4m3_encode(row[k] / sn)) : uint8_t(0);
+    }
+  });
+  return 0;
+}
+
+// FP8 weight tier reference linear: w_hat[n][k] = e4m3(code) * s_n, summed
+// against the bf16 X in fp64.
+int ora_linear_fp8(const uint8_t* codes, const float* row_scales, const uint16_t* x_bf16,
+                   int64_t M, int64_t N, int64_t K, const int64_t* rows, int64_t nrows,
+                   double* y, double* absdot, int nthreads) {
+  if (M < 0 || N < 0 || K < 0 || nrows < 0) return -1;
+  if (!rows && nrows != N) return -1;
+  if (nrows == 0 || M == 0) return 0;
+  if (!y || !row_scales || (K > 0 && (!codes || !x_bf16))) return -1;
+  if (rows)
+    for (int64_t i = 0; i < nrows; ++i)
+      if (rows[i] < 0 || rows[i] >= N) return -1;
+  std::vector<double> xv(size_t(M * K));
+  for (int64_t i = 0; i < M * K; ++i) xv[size_t(i)] = ora_bf16_value(x_bf16[i]);
+  split_range(nrows, nthreads, [&](int64_t lo, int64_t hi) {
+    for (int64_t i = lo; i < hi; ++i) {
+      const int64_t n = rows ? rows[i] : i;
+      const double sn = double(row_scales[n]);
+      for (int64_t m = 0; m < M; ++m) {
+        double sum = 0.0, asum = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+          const double prod = ora_e4m3_decode(codes[n * K + k]) * sn * xv[size_t(m * K + k)];
+          sum += prod;
+          asum += std::fabs(prod);
+        }
+        y[m * nrows + i] = sum;
+        if (absdot) absdot[m * nrows + i] = asum;
+      }
+    }
+  });
+  return 0;
+}
+
 double ora_bytes_model(int64_t M, int64_t N, int64_t K) {
   return double(N) * double(K) / 2.0 + double(N) * double(K) / 16.0 +
          2.0 * double(M) * double(K) + 2.0 * double(M) * double(N);

@@ -18,6 +18,11 @@
  *     Inference Endpoint", section "Recipe (NVIDIA ModelOpt)": weights are
  *     NVFP4 with 16-element scale groups; section "Serving": the checkpoint
  *     keeps the 4-bit codes packed two to a byte (uint8 tensors).
+ *   - The reference linear Y[M,N] = X[M,K] * W^T with W dequantised exactly and
+ *     the sum accumulated in fp64. Page "InventDB Sparkle", section "How it
+ *     answers quickly" (decode reads every weight once per token; the
+ *     guess-and-check scheme verifies several drafted tokens in one pass, so
+ *     M = 1..16).
  *   - Two epilogues of that linear: the SiLU-gated output of a fused gate+up
  *     projection (page "SparkInfer" README, section "Layout & scoring": the
  *     engine's FFN kernels are fused; page "Qwen3.8-27B-NVFP4-RTX5090 API &
@@ -27,11 +32,13 @@
  *     "Qwen3.8-27B-NVFP4-RTX5090 API & Inference Endpoint", section
  *     "SparkInfer + DSpark": a verify pass keeps a drafted token only where it
  *     equals the target's own choice, and near ties at the top can flip).
- *   - The reference linear Y[M,N] = X[M,K] * W^T with W dequantised exactly and
- *     the sum accumulated in fp64. Page "InventDB Sparkle", section "How it
- *     answers quickly" (decode reads every weight once per token; the
- *     guess-and-check scheme verifies several drafted tokens in one pass, so
- *     M = 1..16).
+ *   - Two more tiers of the same linear: W4A4, where X is NVFP4 too (page
+ *     "Qwen3.8-27B-NVFP4-RTX5090 API & Inference Endpoint", section "Recipe
+ *     (NVIDIA ModelOpt)": weights and activations NVFP4 W4A4, group size 16,
+ *     with a per-layer input scale), and 8-bit E4M3 weights as the comparison
+ *     tier (page "InventDB Sparkle", section "How it answers quickly": 8-bit
+ *     weights; same model card, section "Measured against the other NVFP4
+ *     builds of this model": the FP8 tier costs 1.5-2.1x on these shapes).
  *
  * Readings taken where the pages are silent (each is also stated where it is used):
  *   R1 nibble order: element 2j of a row is the low nibble of byte j.
@@ -47,6 +54,12 @@
  *   R11 a fused gate+up projection interleaves its rows: row 2c is the gate
  *      and row 2c+1 the up row of output column c; the gated output is
  *      silu(gate) * up (the SiLU-gated MLP of the model family).
+ *   R14 W4A4: activations are NVFP4 like the weights (16-element blocks of a
+ *      token row, E4M3 block scales) under their own per-tensor scale, which
+ *      the caller gives (a calibrated input scale; synthetic inputs use
+ *      amax(|X|)/(6*448) of the call's X); the same quantiser steps as W.
+ *   R15 FP8 weight tier: E4M3 codes with one fp32 scale per output row,
+ *      s_n = amax(|W[n]|)/448.
  *
  * Parity pins: every function here is pinned by tests under tests/ that do not
  * call back into the same code path (exhaustive tables, brute force, closed
@@ -131,6 +144,31 @@ int ora_swiglu_linear(const uint8_t* packed, const uint8_t* scales, float gs,
  * equal values by ascending index (reading R10); idx is [M][k]. k = 1 is the
  * greedy argmax. Returns 0, -1 on bad arguments, -3 if y holds a NaN. */
 int ora_topk(const double* y, int64_t M, int64_t N, int64_t k, int64_t* idx);
+
+/* W4A4 reference linear (reading R14): X is NVFP4 too, given as x_packed
+ * [M][K/2], x_scales [M][K/16] and its per-tensor scale gs_x (quantise it with
+ * ora_quantize_rows under that scale). y[m*nrows + i] = sum_k w_hat[rows[i]][k]
+ * * x_hat[m][k] in fp64, both operands dequantised exactly; absdot nullable.
+ * Row selection as in ora_linear. Returns 0, or -1 on bad arguments. */
+int ora_linear_w4a4(const uint8_t* w_packed, const uint8_t* w_scales, float gs_w,
+                    const uint8_t* x_packed, const uint8_t* x_scales, float gs_x,
+                    int64_t M, int64_t N, int64_t K, const int64_t* rows, int64_t nrows,
+                    double* y, double* absdot, int nthreads);
+
+/* FP8 weight tier (reading R15): per output row n, s_n = amax(|W[n]|)/448 in
+ * fp32 and codes[n][k] = E4M3(w[n][k] / s_n) (RNE, saturating; the sign of a
+ * negative value that rounds to zero is kept, 0x80); s_n = 0 gives zero codes.
+ * codes is uint8 [N][K], row_scales fp32 [N]. Returns 0, -1 on bad arguments,
+ * -2 if W is not finite. */
+int ora_quantize_fp8_rows(const float* w, int64_t N, int64_t K, uint8_t* codes,
+                          float* row_scales, int nthreads);
+
+/* FP8 weight tier reference linear: y[m*nrows + i] = sum_k e4m3(codes[n][k])
+ * * s_n * x[m][k] in fp64 (n = rows[i]); absdot nullable; rows as in
+ * ora_linear. Returns 0, or -1 on bad arguments. */
+int ora_linear_fp8(const uint8_t* codes, const float* row_scales, const uint16_t* x_bf16,
+                   int64_t M, int64_t N, int64_t K, const int64_t* rows, int64_t nrows,
+                   double* y, double* absdot, int nthreads);
 
 /* Round an fp64 value to bf16 (round to nearest even, overflow to inf), as bits. */
 uint16_t ora_bf16_rne(double v);

@@ -47,6 +47,15 @@ MUTANTS = {
     "top-k ties to the highest index": (
         "(row[a] == row[b] && a < b)",
         "(row[a] == row[b] && a > b)"),
+    "W4A4 drops the activation scale": (
+        "ora_dequant_f64(x_packed, x_scales, gs_x, M, K, xhat.data());",
+        "ora_dequant_f64(x_packed, x_scales, 1.0f, M, K, xhat.data());"),
+    "FP8 row scale over 256 instead of 448": (
+        "const float sn = amax / 448.0f;",
+        "const float sn = amax / 256.0f;"),
+    "FP8 linear drops the row scale": (
+        "ora_e4m3_decode(codes[n * K + k]) * sn * xv[size_t(m * K + k)];",
+        "ora_e4m3_decode(codes[n * K + k]) * xv[size_t(m * K + k)];"),
     "last product of each row dropped": (
         "for (int64_t k = 0; k < K; ++k) {\n          double p",
         "for (int64_t k = 0; k < K - 1; ++k) {\n          double p"),

@@ -497,3 +497,100 @@ def test_argmax_decided_uses_both_bounds():
     assert list(dec) == [True, False, False, True]
     idx1, dec1 = oracle.argmax_decided(np.array([[4.0]]), np.array([[1.0]]))
     assert list(idx1) == [0] and list(dec1) == [True]
+
+
+# ----- tiers: W4A4 and FP8 weights ----------------------------------------
+
+def _random_nvfp4(rows, K, rng, scale_codes=(0x30, 0x38, 0x40, 0x44)):
+    codes = rng.integers(0, 16, size=(rows, K)).astype(np.uint8)
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    scales = rng.choice(np.array(scale_codes, np.uint8), size=(rows, K // 16))
+    return packed, scales
+
+
+def test_w4a4_with_x_on_the_grid_equals_the_bf16_linear():
+    """gs_x = 1/8: each x_hat = e2m1 * e4m3 / 8 is a bf16 value, so the W4A4
+    linear must equal the bf16-X linear on those values, bit for bit."""
+    rng = np.random.default_rng(11)
+    wl = synth.WORKLOADS["tiny"]
+    p, s, gs = oracle.quantize(synth.weights_f32(wl))
+    M = 4
+    xp, xs = _random_nvfp4(M, wl.K, rng)
+    xhat = independent_dequant(xp, xs, 0.125, M, wl.K)
+    X = np.array([[torch_bf16_bits(v) for v in row] for row in xhat], np.uint16)
+    assert np.array_equal(oracle.bf16_bits_to_f64(X), xhat)      # on the bf16 grid
+    y4, ad4 = oracle.linear_w4a4(p, s, gs, xp, xs, 0.125, M, wl.N, wl.K)
+    y, ad = oracle.linear(p, s, gs, X, M, wl.N, wl.K)
+    assert np.array_equal(y4, y) and np.array_equal(ad4, ad)
+
+
+def test_w4a4_matches_independent_construction():
+    wl = synth.WORKLOADS["tiny"]
+    p, s, gs = oracle.quantize(synth.weights_f32(wl))
+    M = 3
+    X = synth.x_bf16_custom(synth.X_OUTLIERS, M, wl.K, seed=2, n_outliers=4, gain=20.0)
+    xp, xs, gs_x = oracle.quantize_x(X)
+    x = oracle.bf16_bits_to_f64(X)
+    assert gs_x == float(np.float32(np.abs(x).max()) / np.float32(2688.0))
+    xhat = independent_dequant(xp, xs, gs_x, M, wl.K)
+    W = independent_dequant(p, s, gs, wl.N, wl.K)
+    y, ad = oracle.linear_w4a4(p, s, gs, xp, xs, gs_x, M, wl.N, wl.K)
+    assert np.allclose(y, xhat @ W.T, rtol=1e-12, atol=1e-15)
+    assert np.allclose(ad, np.abs(xhat) @ np.abs(W).T, rtol=1e-12)
+    rows = np.array([3, 511, 0])
+    yr, _ = oracle.linear_w4a4(p, s, gs, xp, xs, gs_x, M, wl.N, wl.K, rows=rows)
+    assert np.array_equal(yr, y[:, rows])
+    # each x_hat is within half an E2M1 step of x (steps are <= half the
+    # magnitude, or d/2 near zero, d = decoded block scale * gs_x)
+    d = np.repeat(np.vectorize(torch_e4m3_value)(xs), 16, axis=1) * gs_x
+    assert np.all(np.abs(xhat - x) <= 0.25 * (np.abs(x) + d))
+
+
+def test_fp8_rows_match_torch_e4m3():
+    rng = np.random.default_rng(13)
+    w = (rng.normal(0.0, 0.02, size=(64, 96)) * rng.uniform(0.1, 10.0, size=(64, 1))).astype(np.float32)
+    w[5] = 0.0
+    w[7, 3] = -1e-12                                       # rounds to zero, keeps its sign
+    codes, sc = oracle.quantize_fp8_rows(w)
+    amax = np.abs(w).max(axis=1)
+    assert np.array_equal(sc, amax / np.float32(448.0))
+    assert sc[5] == 0.0 and not codes[5].any()
+    live = sc > 0
+    u = (w[live] / sc[live, None]).astype(np.float32)
+    ref = torch.from_numpy(u).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes[live], ref)
+    assert codes[7, 3] == 0x80
+    with pytest.raises(ValueError):
+        oracle.quantize_fp8_rows(np.array([[1.0, float("inf")]], np.float32))
+
+
+def test_fp8_round_trip_on_grid():
+    """Rows of E4M3 values times 2^j that hold +-448 * 2^j quantise back to
+    the same codes under s_n = 2^j."""
+    rng = np.random.default_rng(17)
+    N, K = 16, 64
+    codes = rng.integers(1, 0x7F, size=(N, K)).astype(np.uint8)
+    codes |= (rng.integers(0, 2, size=(N, K)) << 7).astype(np.uint8)
+    codes[:, 0] = 0x7E                                      # 448
+    vals = np.vectorize(torch_e4m3_value)(codes)
+    pw = 2.0 ** rng.integers(-12, 4, size=(N, 1))
+    w = (vals * pw).astype(np.float32)
+    got, sc = oracle.quantize_fp8_rows(w)
+    assert np.array_equal(sc.astype(np.float64), pw[:, 0])
+    assert np.array_equal(got, codes)
+
+
+def test_fp8_linear_matches_independent_matmul():
+    rng = np.random.default_rng(19)
+    N, K, M = 40, 128, 3
+    w = rng.normal(0.0, 0.05, size=(N, K)).astype(np.float32)
+    codes, sc = oracle.quantize_fp8_rows(w)
+    X = synth.x_bf16_custom(synth.X_NORMAL, M, K, seed=6)
+    x = oracle.bf16_bits_to_f64(X)
+    W = np.vectorize(torch_e4m3_value)(codes) * sc.astype(np.float64)[:, None]
+    y, ad = oracle.linear_fp8(codes, sc, X, M, N, K)
+    assert np.allclose(y, x @ W.T, rtol=1e-12, atol=1e-15)
+    assert np.allclose(ad, np.abs(x) @ np.abs(W).T, rtol=1e-12)
+    rows = np.array([39, 0, 12])
+    yr, _ = oracle.linear_fp8(codes, sc, X, M, N, K, rows=rows)
+    assert np.array_equal(yr, y[:, rows])
