@@ -85,6 +85,11 @@ class ClockSampler:
         time.sleep(0.2)
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
+        return self.summarize(out)
+
+    def summarize(self, out: str):
+        """Median SM clock, max clock and the throttle reasons seen Active in
+        the samples inside the timed region [t0, t1] (60 ms margin)."""
         import datetime
         rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
         sm, smax, reasons, total = [], None, set(), 0

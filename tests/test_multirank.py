@@ -144,3 +144,30 @@ def test_reference_arm_prints_the_contract_line():
     assert d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert "workload" in d["config"]
+
+
+def test_clock_sampler_keeps_timed_region_and_active_reasons():
+    """Host logic of the clocks record: only samples inside the timed region
+    count, and a throttle reason is reported when any of them shows it Active."""
+    import datetime
+    import bench
+    t0 = datetime.datetime(2026, 1, 1, 12, 0, 0).timestamp()
+
+    def row(dt, mhz, reasons=("Not Active",) * 4):
+        ts = datetime.datetime.fromtimestamp(t0 + dt).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return ", ".join([ts, "0", str(mhz), "1965", "900.5", "0x0"] + list(reasons))
+
+    out = "\n".join([
+        row(-1.0, 600, ("Active", "Not Active", "Not Active", "Not Active")),  # before: ignored
+        row(0.1, 1800),
+        row(0.2, 1900, ("Not Active", "Not Active", "Not Active", "Active")),
+        row(0.3, 1950),
+        "garbage line",
+        row(5.0, 300, ("Not Active", "Active", "Not Active", "Not Active")),   # after: ignored
+    ])
+    cs = bench.ClockSampler(0)
+    cs.t0, cs.t1 = t0, t0 + 0.5
+    d = cs.summarize(out)
+    assert d["sm_mhz"] == 1900 and d["sm_max_mhz"] == 1965
+    assert d["reasons"] == ["sw_power_cap"]
+    assert d["samples"] == 3 and d["samples_total"] == 5
