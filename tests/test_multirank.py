@@ -171,3 +171,24 @@ def test_clock_sampler_keeps_timed_region_and_active_reasons():
     assert d["sm_mhz"] == 1900 and d["sm_max_mhz"] == 1965
     assert d["reasons"] == ["sw_power_cap"]
     assert d["samples"] == 3 and d["samples_total"] == 5
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """Two ranks launched by torchrun: rank 0 alone runs the oracle and prints
+    one line, the other rank exits 0 without work."""
+    import json
+    import socket
+    import subprocess
+    import sys
+    from tests.conftest import ROOT
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "2", "--master-addr", "127.0.0.1", "--master-port",
+                        str(port), "bench.py", "--gpus", "2", "--impl", "reference", "--steps", "1",
+                        "--warmup", "0", "--reference-rows", "128"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
