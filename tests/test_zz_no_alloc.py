@@ -6,7 +6,6 @@ one finds the first one's leftovers in the shared array).
 Collected last on purpose: it must pass in a fresh process and after every
 other test has used the device.
 """
-import numpy as np
 import pytest
 import torch
 
