@@ -37,7 +37,10 @@ _LIB = os.path.join(_HERE, "libnvfp4_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-NTHREADS = max(1, os.cpu_count() or 1)
+# host threads: the cores this process may run on (its affinity mask), which
+# can be fewer than the machine's
+NTHREADS = max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity")
+               else (os.cpu_count() or 1))
 
 
 def build(force: bool = False) -> str:

@@ -35,7 +35,10 @@ _SRC = os.path.join(_HERE, "synth.cpp")
 _LIB = os.path.join(_HERE, "libsynth.so")
 _lock = threading.Lock()
 _lib = None
-NTHREADS = max(1, os.cpu_count() or 1)
+# host threads: the cores this process may run on (its affinity mask), which
+# can be fewer than the machine's
+NTHREADS = max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity")
+               else (os.cpu_count() or 1))
 
 X_NORMAL, X_OUTLIERS, X_SWIGLU, X_RMSNORM = 0, 1, 2, 3
 
