@@ -470,6 +470,11 @@ def run_ours(args):
 # ---------------------------------------------------------------------------
 
 def run_reference(args):
+    """The oracle as it stands, timed on the host cores over `steps` calls
+    after `warmup` calls, each call on a row sample of the workload. The
+    sample is sized so that the whole run takes about --reference-budget
+    seconds (unless --reference-rows fixes it); `cores` reports the threads
+    the oracle actually used for that sample."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
@@ -477,25 +482,43 @@ def run_reference(args):
     import synth
     wl = synth.WORKLOADS[args.workload]
     M = args.M
-    rows = max(64, min(wl.N, int(args.reference_rows)))
-    gs = oracle.global_scale(synth.weights_f32(wl))
-    packed, scales = oracle.quantize_rows(synth.weights_f32(wl, rows=slice(0, rows)), gs)
     X = synth.x_bf16(wl, M)
-    cores = oracle.NTHREADS
+    gs = oracle.global_scale(synth.weights_f32(wl))
+    calls = max(1, args.steps) + max(0, args.warmup)
+    if args.reference_rows:
+        rows = max(1, min(wl.N, int(args.reference_rows)))
+    else:
+        # untimed calibration: seconds per row on one thread
+        cal = 256
+        p, s = oracle.quantize_rows(synth.weights_f32(wl, rows=slice(0, cal)), gs)
+        t0 = time.perf_counter()
+        oracle.linear(p, s, gs, X, M, cal, wl.K, nthreads=1)
+        per_row = (time.perf_counter() - t0) / cal
+        per_call = args.reference_budget / calls
+        par_min = next(n for n in (2 ** i for i in range(40)) if oracle.threads_for(n) > 1) \
+            if oracle.NTHREADS > 1 else None
+        par_rows = int(per_call * oracle.NTHREADS / per_row)
+        if par_min is not None and par_rows >= par_min:
+            rows = min(wl.N, par_rows)                   # large enough to use every core
+        else:
+            rows = min(wl.N, (par_min or wl.N + 1) - 1, max(16, int(per_call / per_row)))
+    cores = oracle.threads_for(rows)
+    packed, scales = oracle.quantize_rows(synth.weights_f32(wl, rows=slice(0, rows)), gs)
     for _ in range(max(0, args.warmup)):
-        oracle.linear(packed, scales, gs, X, M, rows, wl.K, nthreads=cores)
+        oracle.linear(packed, scales, gs, X, M, rows, wl.K)
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle.linear(packed, scales, gs, X, M, rows, wl.K, nthreads=cores)
+    for _ in range(max(1, args.steps)):
+        oracle.linear(packed, scales, gs, X, M, rows, wl.K)
     sec = (time.perf_counter() - t0) / max(1, args.steps)
     value = effective_gbs(bytes_per_call(M, rows, wl.K), sec)
     sample = ("each step: fp64 oracle linear on the first %d of %d rows of the %s workload "
-              "(M=%d, K=%d), bytes scaled to the sample" % (rows, wl.N, args.workload, M, wl.K))
+              "(M=%d, K=%d) on %d host thread(s), bytes scaled to the sample"
+              % (rows, wl.N, args.workload, M, wl.K, cores))
     line = {
         # n_gpus is the launch's world size; the oracle itself runs on rank 0's host cores only
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "steps": max(1, args.steps), "warmup": args.warmup, "ms_per_step": sec * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
         "config": {"workload": "%s projection M=%d K=%d N=%d" % (args.workload, M, wl.K, wl.N),
@@ -522,7 +545,10 @@ def main():
     ap.add_argument("--full-sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--reference-rows", type=int, default=2048)
+    ap.add_argument("--reference-rows", type=int, default=0,
+                    help="rows of the workload per reference call (0: sized from the budget)")
+    ap.add_argument("--reference-budget", type=float, default=90.0,
+                    help="seconds the reference arm's warm-up and timed calls should take")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

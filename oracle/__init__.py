@@ -65,6 +65,7 @@ def _load():
         c = ctypes
         P = c.c_void_p
         sig = {
+            "ora_threads_for": (c.c_int, [c.c_int64, c.c_int]),
             "ora_e2m1_decode": (c.c_double, [c.c_uint32]),
             "ora_e4m3_decode": (c.c_double, [c.c_uint32]),
             "ora_e4m3_is_nan": (c.c_int, [c.c_uint32]),
@@ -106,6 +107,11 @@ def _ptr(a):
 def _c(a, dtype):
     a = np.ascontiguousarray(a, dtype=dtype)
     return a
+
+
+def threads_for(nrows: int, nthreads: int = NTHREADS) -> int:
+    """Host threads the row-parallel oracle functions use for `nrows` rows."""
+    return int(_load().ora_threads_for(int(nrows), int(nthreads)))
 
 
 # ---- scalar codecs -------------------------------------------------------

@@ -16,11 +16,15 @@
 
 namespace {
 
-// Run body(lo, hi) over [0, n) split into nthreads contiguous pieces.
+// Ranges shorter than this run on the calling thread alone.
+constexpr int64_t kParallelMin = 4096;
+
+// Run body(lo, hi) over [0, n) split into nthreads contiguous pieces
+// (ora_threads_for(n, nthreads) of them are non-empty).
 template <class F>
 void split_range(int64_t n, int nthreads, F body) {
   if (nthreads < 1) nthreads = 1;
-  if (n < 4096 || nthreads == 1) { body(int64_t(0), n); return; }
+  if (n < kParallelMin || nthreads == 1) { body(int64_t(0), n); return; }
   int64_t per = (n + nthreads - 1) / nthreads;
   std::vector<std::thread> ts;
   for (int t = 0; t < nthreads; ++t) {
@@ -59,6 +63,13 @@ int nearest_even(const double* table, int n, double a) {
 }  // namespace
 
 extern "C" {
+
+int ora_threads_for(int64_t n, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  if (n < kParallelMin || nthreads == 1) return 1;
+  const int64_t per = (n + nthreads - 1) / nthreads;
+  return int((n + per - 1) / per);
+}
 
 // OCP Microscaling spec, E2M1: sign bit 3, exponent bits 2..1 (bias 1),
 // mantissa bit 0; exponent 0 is subnormal with value m * 0.5.

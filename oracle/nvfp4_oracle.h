@@ -74,6 +74,11 @@
 extern "C" {
 #endif
 
+/* Host threads the row-parallel functions (quantiser, linears) use for n rows
+ * when given nthreads: 1 below 4096 rows, else the number of non-empty
+ * contiguous pieces. */
+int ora_threads_for(int64_t n, int nthreads);
+
 /* Value of an E2M1 code (low 4 bits used). Code 0x8 decodes to -0.0. */
 double ora_e2m1_decode(uint32_t code);
 /* Value of an E4M3 ("fn") byte. 0x7F and 0xFF decode to NaN. */

@@ -192,3 +192,38 @@ def test_reference_arm_under_torchrun_prints_once():
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [json.loads(l) for l in r.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+
+
+def test_oracle_thread_count_helper():
+    """Documented values: one thread below 4096 rows, else the non-empty
+    contiguous pieces of the split, never more than asked for."""
+    import oracle
+    assert oracle.threads_for(0, 8) == 1 and oracle.threads_for(4095, 64) == 1
+    assert oracle.threads_for(10 ** 6, 1) == 1
+    for n in (4096, 4097, 5000, 34816, 248320):
+        for t in (2, 3, 8, 16, 64):
+            k = oracle.threads_for(n, t)
+            per = -(-n // t)
+            assert 1 < k <= t and (k - 1) * per < n <= k * per
+
+
+def test_reference_arm_sizes_its_sample_to_the_budget():
+    """With no fixed row count the reference arm sizes each call from the time
+    budget and reports the threads the oracle used for that sample."""
+    import json
+    import re
+    import subprocess
+    import sys
+    import time
+    import oracle
+    from tests.conftest import ROOT
+    t0 = time.time()
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "300",
+                          "--warmup", "3", "--reference-budget", "3"], cwd=ROOT,
+                         capture_output=True, text=True, timeout=600, check=True).stdout
+    wall = time.time() - t0
+    d = json.loads([l for l in out.splitlines() if l.startswith("{")][0])
+    rows = int(re.search(r"first (\d+) of", d["cpu_baseline"]["sample"]).group(1))
+    assert d["cpu_baseline"]["cores"] == oracle.threads_for(rows)
+    assert d["steps"] == 300 and d["ms_per_step"] * 303 < 3 * 1000 * 3   # within 3x the budget
+    assert wall < 120
