@@ -340,12 +340,12 @@ def cpu_baseline(sample_rows: int = 34816, M: int = 1):
     gs = oracle.global_scale(synth.weights_f32(wl))
     packed, scales = oracle.quantize_rows(W, gs)
     X = synth.x_bf16(wl, M)
-    cores = oracle.NTHREADS
-    oracle.linear(packed, scales, gs, X, M, rows, wl.K, nthreads=cores)   # warm-up
+    cores = oracle.threads_for(rows, oracle.NTHREADS)    # threads the oracle uses here
+    oracle.linear(packed, scales, gs, X, M, rows, wl.K, nthreads=oracle.NTHREADS)   # warm-up
     ts = []
     for _ in range(3):
         t0 = time.perf_counter()
-        oracle.linear(packed, scales, gs, X, M, rows, wl.K, nthreads=cores)
+        oracle.linear(packed, scales, gs, X, M, rows, wl.K, nthreads=oracle.NTHREADS)
         ts.append(time.perf_counter() - t0)
     t = statistics.median(ts)
     return {"value": effective_gbs(bytes_per_call(M, rows, wl.K), t), "unit": "GB/s",
