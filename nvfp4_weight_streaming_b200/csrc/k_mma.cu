@@ -27,7 +27,8 @@
 //
 // B is X in f16, scaled per token by a power of two (largest magnitude at
 // 2^14) in a hi plane (exact within 2^28 of that maximum) and a lo plane
-// scaled by 2^29 (the next 29 binades); elements further below are dropped.
+// scaled by 2^29 (exact for the next 29 binades); elements further below keep
+// only the lo plane's subnormal step (within 2^-68 of the maximum).
 // Columns are groups of 64 elements padded to 136 bytes, so B fragments are
 // bank-conflict-free 8-byte shared loads at immediate offsets. Every product
 // is exact; only the fp32 accumulation rounds. When no element needs the lo
@@ -227,10 +228,6 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
   }
 }
 
-// One step of one lane: decode rows r and r+8 of the stage (64 elements each)
-// and issue the MMAs for NTILE 8-column token tiles. MMA i of the step adds
-// into accumulator set i % (4 / NTILE): four independent chains per warp,
-// instead of sixteen MMAs serialised on one accumulator.
 // Largest bf16 magnitude (bits, sign cleared) among the eight values of a
 // 16-byte chunk, with one packed 16-bit max per pair.
 __device__ __forceinline__ uint32_t bf16_mag_max8(const uint4& v) {
@@ -321,6 +318,11 @@ k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ plan
   }
 }
 
+// One step of one lane: decode rows r and r+8 of the stage (64 elements each)
+// and issue the MMAs for NTILE 8-column token tiles. MMA i of the step adds
+// into accumulator set i % (4 / NTILE): four independent chains per warp,
+// instead of sixteen MMAs serialised on one accumulator. PRED: token tiles
+// flagged off in `xon` read a zero B fragment instead of shared memory.
 // EARLY: after loading its share of the stage into registers the warp
 // releases the slot (lane 0 arrives on `empty`), so the refill overlaps the
 // decode and the MMAs.
