@@ -26,8 +26,9 @@
 // that the token's largest magnitude sits at 2^14, in two planes: "hi" holds
 // every element within 2^28 of that maximum exactly (bf16 has 8 significant
 // bits, f16 normals 11), "lo" holds the elements 2^28..2^57 below it, scaled up
-// by 2^29. Elements further below are dropped. Every product is then exact in
-// fp32 and only the fp32 accumulation rounds.
+// by 2^29. Elements further below keep only the lo plane's subnormal step
+// (within 2^-68 of the maximum). Every product is then exact in fp32 and only
+// the fp32 accumulation rounds.
 //
 // Work split. K is cut into S slices (so that a slice of X fits in shared
 // memory); the CTAs of a slice share its (tile, k-step) space evenly (stream-K).
