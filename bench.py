@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "NVFP4 linear effective HBM GB/s and % of peak at M=1/16 (27B-class shapes)"
 NOMINAL_HBM_GBS = 8000.0
+VARIANT_NAMES = ("auto", "gemv", "mma", "tc", "row")
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -391,7 +392,7 @@ def run_ours(args):
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
     peak, peak_kind = peaks()
-    variant = {"auto": 0, "gemv": 1, "mma": 2, "tc": 3}[args.variant]
+    variant = {"auto": 0, "gemv": 1, "mma": 2, "tc": 3, "row": 4}[args.variant]
     flags = 0 if args.no_pdl else nv.NVFP4_PLAN_PDL
     pb = Problem(args.workload, args.M, variant, min_footprint=4.2 * l2, flags=flags)
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
@@ -411,7 +412,7 @@ def run_ours(args):
             s2, _ = time_problem(q, max(args.steps, 200), args.warmup, world)
             g = effective_gbs(q.bytes, s2)
             sweep.append({"workload": name, "M": M, "N": q.N, "K": q.K,
-                          "variant": ["auto", "gemv", "mma", "tc"][q.variant],
+                          "variant": VARIANT_NAMES[q.variant],
                           "split_k": q.split_k, "us_per_call": s2 * 1e6, "GBps": g,
                           "frac_of_measured_peak": g / peak})
             q.destroy()
@@ -434,7 +435,7 @@ def run_ours(args):
             "data": "synthetic (seeded SplitMix64/Box-Muller, workload recipes in synth/)",
             "config": {"workload": "%s projection M=%d K=%d N=%d" % (args.workload, pb.M, pb.K, pb.N),
                        "M": pb.M, "K": pb.K, "N": pb.N,
-                       "variant": ["auto", "gemv", "mma", "tc"][pb.variant],
+                       "variant": VARIANT_NAMES[pb.variant],
                        "split_k": pb.split_k, "bytes_per_call": pb.bytes,
                        "l2": "inputs larger than L2: %d byte-identical weight copies "
                              "rotated, %.0f MB > %.1f x %.0f MB L2" %
@@ -448,7 +449,7 @@ def run_ours(args):
             "pct_of_nominal_8TBps": 100 * per_gpu / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s",
                          "frac": per_gpu / peak,
-                         "traffic": measured_traffic(["auto", "gemv", "mma", "tc"][pb.variant],
+                         "traffic": measured_traffic(VARIANT_NAMES[pb.variant],
                                                      "%s projection M=%d K=%d N=%d" %
                                                      (args.workload, pb.M, pb.K, pb.N)),
                          "peak_kind": peak_kind + " device-copy bandwidth (MEASURED_PEAKS hbm_gbs)"},
@@ -538,7 +539,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode")
     ap.add_argument("--M", type=int, default=1)
-    ap.add_argument("--variant", choices=["auto", "gemv", "mma", "tc"], default="auto")
+    ap.add_argument("--variant", choices=list(VARIANT_NAMES), default="auto")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch")

@@ -28,7 +28,15 @@
  * contraction accumulates in fp32 (tensor cores or CUDA cores, by variant);
  * the epilogue computes y = gs * acc in fp32 and rounds to bf16 (nearest even).
  * Per element |y - y_ref| <= 1e-2 |y_ref| + 1e-4 sum_k |w_hat x| against an
- * fp64 reference.
+ * fp64 reference, for every X whose rows keep each nonzero element within
+ * 2^57 of the row's largest magnitude. The tensor-core variants take X as
+ * f16: each token row is scaled by a power of two (largest magnitude at
+ * 2^14) and split into a hi plane and a lo plane (scaled by 2^29), which
+ * together hold every such element exactly. An element further below its
+ * row maximum keeps only the lo plane's subnormal step (absolute error at
+ * most 2^-68 max_k |x[m][k]|), so for rows that hold one the bound above
+ * gains the term 2^-67 max_k |x[m][k]| sum_k |w_hat[n][k]|. The CUDA-core
+ * variant (GEMV) has no such range condition.
  *
  * Conventions.
  *   - Every buffer is device memory owned by the caller; the library never
@@ -70,14 +78,17 @@ typedef enum {
 
 typedef struct nvfp4_plan_s* nvfp4_plan_t;
 
-/* Kernel variants (plan flags, bits 0..3). AUTO takes MMA, the fastest on
- * B200 for every M measured, and TC for a shape MMA cannot take. */
+/* Kernel variants (plan flags, bits 0..3). AUTO takes the variant measured
+ * fastest on B200 for the plan's (M, N, K), and TC for a shape the chosen
+ * variant cannot take. */
 #define NVFP4_VARIANT_AUTO 0u
 #define NVFP4_VARIANT_GEMV 1u  /* CUDA-core warp-per-row GEMV, fp32 FMA        */
 #define NVFP4_VARIANT_MMA  2u  /* TMA ring + warp MMA (m16n8k16), stream-K    */
 #define NVFP4_VARIANT_TC   3u  /* tcgen05 + TMA ring + TMEM accumulators       */
+#define NVFP4_VARIANT_ROW  4u  /* M <= 2: 16-row units taken dynamically, warp
+                                  MMA with a block-diagonal X operand          */
 #define NVFP4_PLAN_VARIANT_MASK 0xFu
-/* Programmatic dependent launch (MMA variant; ignored by the others). The
+/* Programmatic dependent launch (MMA and ROW variants; ignored by the others). The
  * launch may start while the previous kernel in the stream is still running:
  * it begins streaming W at once and touches X, Y, w_global and the workspace
  * only after that kernel has completed. So W (codes and scales) must not be

@@ -20,6 +20,7 @@ __all__ = [
     "NVFP4_OK", "NVFP4_ERR_INVALID_ARG", "NVFP4_ERR_UNSUPPORTED", "NVFP4_ERR_MISALIGNED",
     "NVFP4_ERR_CUDA", "NVFP4_ERR_TIMEOUT", "NVFP4_ERR_BAD_SCALE", "NVFP4_ERR_WORKSPACE",
     "NVFP4_VARIANT_AUTO", "NVFP4_VARIANT_GEMV", "NVFP4_VARIANT_MMA", "NVFP4_VARIANT_TC",
+    "NVFP4_VARIANT_ROW",
     "NVFP4_PLAN_PDL", "NVFP4_PLAN_TEST_STALL",
     "Nvfp4Error", "lib", "library_path",
     "nvfp4_linear_plan", "nvfp4_linear_workspace_bytes", "nvfp4_linear_variant",
@@ -42,6 +43,7 @@ NVFP4_VARIANT_AUTO = 0
 NVFP4_VARIANT_GEMV = 1
 NVFP4_VARIANT_MMA = 2
 NVFP4_VARIANT_TC = 3
+NVFP4_VARIANT_ROW = 4
 NVFP4_PLAN_PDL = 0x10000
 NVFP4_PLAN_TEST_STALL = 0x40000000
 NVFP4_STATIC_SCRATCH_BYTES = 16 << 20

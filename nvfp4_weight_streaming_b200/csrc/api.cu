@@ -37,6 +37,7 @@ struct nvfp4_plan_s {
   nvfp4::GemvConfig gemv;
   nvfp4::TcConfig tc;
   nvfp4::MmaConfig mma;
+  nvfp4::RowConfig row;
   std::mutex map_mu;
   MapEntry maps[kMapCache];
   int map_next = 0;
@@ -80,8 +81,8 @@ nvfp4_status static_scratch_address(int device, void** out) {
 // against 105.9 for tcgen05); plan() falls back to tcgen05 for shapes it
 // cannot take.
 int auto_variant(int M, int N, int K) {
-  (void)M; (void)N; (void)K;
-  return int(NVFP4_VARIANT_MMA);
+  (void)N; (void)K;
+  return M <= 2 ? int(NVFP4_VARIANT_ROW) : int(NVFP4_VARIANT_MMA);
 }
 
 // Copy of the TMA descriptors for (wp, ws), encoding them on first use.
@@ -95,9 +96,16 @@ bool lookup_maps(nvfp4_plan_s* p, const void* wp, const void* ws, CUtensorMap* m
     }
   }
   MapEntry& e = p->maps[p->map_next];
-  const int box_rows = p->variant == int(NVFP4_VARIANT_MMA) ? nvfp4::kMmaTileRows : 128;
-  if (!nvfp4::encode_weight_maps(p->N, p->K, box_rows, static_cast<const uint8_t*>(wp),
-                                 static_cast<const uint8_t*>(ws), &e.mw, &e.ms)) {
+  bool ok;
+  if (p->variant == int(NVFP4_VARIANT_ROW)) {
+    ok = nvfp4::encode_row_maps(p->N, p->K, p->row.ipu, static_cast<const uint8_t*>(wp),
+                                static_cast<const uint8_t*>(ws), &e.mw, &e.ms);
+  } else {
+    const int box_rows = p->variant == int(NVFP4_VARIANT_MMA) ? nvfp4::kMmaTileRows : 128;
+    ok = nvfp4::encode_weight_maps(p->N, p->K, box_rows, static_cast<const uint8_t*>(wp),
+                                   static_cast<const uint8_t*>(ws), &e.mw, &e.ms);
+  }
+  if (!ok) {
     e.wp = e.ws = nullptr;
     return false;
   }
@@ -177,6 +185,17 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
         p.ws_bytes = p.mma.ws_bytes;
         break;
       }
+      case NVFP4_VARIANT_ROW: {
+        if (K == 0 || N == 0) break;
+        p.row.M = M; p.row.N = N; p.row.K = K;
+        cudaError_t e = nvfp4::row_configure(p.row, sms);
+        if (e == cudaSuccess && !nvfp4::tensor_maps_supported()) e = cudaErrorNotSupported;
+        if (e == cudaErrorInvalidConfiguration || e == cudaErrorNotSupported) st = NVFP4_ERR_UNSUPPORTED;
+        else if (e != cudaSuccess) st = NVFP4_ERR_CUDA;
+        p.split_k = p.row.KS;
+        p.ws_bytes = p.row.ws_bytes;
+        break;
+      }
       case NVFP4_VARIANT_TC: {
         if (K == 0 || N == 0) break;
         p.tc.M = M; p.tc.N = N; p.tc.K = K;
@@ -193,6 +212,13 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
     return st;
   };
   nvfp4_status st = configure();
+  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.variant == int(NVFP4_VARIANT_ROW)) {
+    // the row variant cannot take this shape (X too large to stay resident)
+    p.variant = int(NVFP4_VARIANT_MMA);
+    p.split_k = 1;
+    p.ws_bytes = 0;
+    st = configure();
+  }
   if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.variant != int(NVFP4_VARIANT_TC)) {
     // the automatic choice cannot take this shape: the tcgen05 pipeline can
     p.variant = int(NVFP4_VARIANT_TC);
@@ -267,6 +293,15 @@ nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
           mx = plan->xmap;
         }
         e = nvfp4::launch_mma(plan->mma, &mw, &ms, &mx, w_global, xb, yb, workspace,
+                              stall ? kStallTimeoutCycles : kTimeoutCycles, stall, pdl, st);
+        break;
+      }
+      case NVFP4_VARIANT_ROW: {
+        CUtensorMap mw, ms;
+        if (!lookup_maps(plan, w_packed, w_scales, &mw, &ms)) return NVFP4_ERR_CUDA;
+        const bool stall = (plan->flags & NVFP4_PLAN_TEST_STALL) != 0;
+        const bool pdl = (plan->flags & NVFP4_PLAN_PDL) != 0;
+        e = nvfp4::launch_row(plan->row, &mw, &ms, w_global, xb, yb, workspace,
                               stall ? kStallTimeoutCycles : kTimeoutCycles, stall, pdl, st);
         break;
       }
@@ -361,6 +396,8 @@ nvfp4_status nvfp4_linear_run_static(nvfp4_plan_t plan, const uint8_t* w_packed,
     zeroed = plan->mma.ws_partials_off;
   if (plan->variant == int(NVFP4_VARIANT_TC) && plan->tc.ws_partials_off < zeroed)
     zeroed = plan->tc.ws_partials_off;
+  if (plan->variant == int(NVFP4_VARIANT_ROW) && plan->row.ws_partials_off < zeroed)
+    zeroed = plan->row.ws_partials_off;
   if (zeroed > 0 && cudaMemsetAsync(scratch, 0, zeroed, st) != cudaSuccess) return NVFP4_ERR_CUDA;
   s = nvfp4_linear_run(plan, w_packed, w_scales, w_global, x, y, scratch,
                        size_t(NVFP4_STATIC_SCRATCH_BYTES), stream);

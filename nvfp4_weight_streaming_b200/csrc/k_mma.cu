@@ -85,7 +85,7 @@ inline int misc_bytes(int M) { return MISC_BASE + (M <= 4 ? M * TROWS * 4 : 0); 
 // piece slots [384,640), end-phase list [640,896)
 constexpr int MISC_EMAX = 256, MISC_FLAGS = 320, MISC_SKIP = 336, MISC_PREFLAG = 368, MISC_PIECES = 384,
               MISC_LIST = 640, MISC_PREBUF = 1024;   // prefetched piece: [M <= 4][TROWS] floats
-constexpr int LO_SHIFT = 29;
+constexpr int LO_SHIFT = X_LO_SHIFT;
 constexpr int BAR_CONSUMERS = 1;           // named barrier of the consumer warps
 constexpr int XR_MIN_M = 5;                // token counts from which X goes through the ring
 
@@ -226,52 +226,6 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
       return;
     }
   }
-}
-
-// Largest bf16 magnitude (bits, sign cleared) among the eight values of a
-// 16-byte chunk, with one packed 16-bit max per pair.
-__device__ __forceinline__ uint32_t bf16_mag_max8(const uint4& v) {
-  const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                              __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
-  return max(m & 0xFFFFu, m >> 16);
-}
-
-// Exponent floor(log2 |x|) of the bf16 magnitude `mag`; INT_MIN for zero.
-__device__ __forceinline__ int bf16_mag_exp(uint32_t mag) {
-  if (mag == 0u) return INT_MIN;
-  const uint32_t e8 = mag >> 7;
-  if (e8) return int(e8) - 127;
-  return (31 - __clz(int(mag & 0x7Fu))) - 133;     // subnormal
-}
-
-// Two bf16 values (one word) -> their hi f16 pair and lo f16 pair for the
-// token's shift: x * 2^sh (exact: the scale is applied as two powers of two
-// f1 * f2) rounded to f16 is the hi plane (exact for |x * 2^sh| >= 2^-14:
-// 8 significant bits), the exact remainder scaled by 2^LO_SHIFT is the lo
-// plane. Returns the lo pair.
-__device__ __forceinline__ uint32_t x_split2(uint32_t w, float f1, float f2, uint32_t& hi) {
-  const float s0 = (__uint_as_float(w << 16) * f1) * f2;
-  const float s1 = (__uint_as_float(w & 0xFFFF0000u) * f1) * f2;
-  const __half2 h = __floats2half2_rn(s0, s1);       // low half = element 0
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  const float2 hb = __half22float2(h);
-  constexpr float kLo = 536870912.0f;                 // 2^LO_SHIFT
-  const __half2 l = __floats2half2_rn((s0 - hb.x) * kLo, (s1 - hb.y) * kLo);
-  return *reinterpret_cast<const uint32_t*>(&l);
-}
-
-// Eight bf16 values (four words) -> hi and lo planes for the token's shift
-// sh (largest magnitude at 2^14); returns whether any lo element is nonzero.
-__device__ __forceinline__ bool x_split8(const uint32_t w[4], int sh, uint32_t hi[4], uint32_t lo[4]) {
-  static_assert(LO_SHIFT == 29, "kLo above is 2^29");
-  const float f1 = __int_as_float((127 + sh / 2) << 23), f2 = __int_as_float((127 + sh - sh / 2) << 23);
-  uint32_t any = 0u;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    lo[q] = x_split2(w[q], f1, f2, hi[q]);
-    any |= lo[q] & 0x7FFF7FFFu;
-  }
-  return any != 0u;
 }
 
 // X in the ring: one CTA per token converts its row of X into the hi and lo

@@ -334,7 +334,7 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
               uint32_t sg;
               const int th = bf16_exp(b, sg) + sh;
               if (th >= -14) hi[i >> 1] |= make_f16(b >> 15, th, sg) << (16 * (i & 1));
-              else lo[i >> 1] |= make_f16(b >> 15, th + LO_SHIFT, sg) << (16 * (i & 1));
+              else lo[i >> 1] |= make_f16_rn(b >> 15, th + LO_SHIFT, sg) << (16 * (i & 1));
             }
           }
           lo_used |= (lo[0] | lo[1] | lo[2] | lo[3]) != 0u;
@@ -682,6 +682,8 @@ bool encode_x_planes_map(const void* planes, int pitch_bytes, int cols, int box_
 }
 
 bool tensor_maps_supported() { return tc::encode_fn() != nullptr; }
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() { return tc::encode_fn(); }
 
 cudaError_t launch_tc(const TcConfig& c, const void* map_w, const void* map_s, const float* gs,
                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,

@@ -4,6 +4,8 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 namespace nvfp4 {
@@ -67,5 +69,26 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
                        const float* gs, const uint16_t* x, uint16_t* y, void* workspace,
                        long long timeout_cycles, bool stall, bool pdl, cudaStream_t st);
 constexpr int kMmaTileRows = 256;
+
+// The driver's cuTensorMapEncodeTiled (null if unavailable); k_tc.cu.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// Row-block streaming variant, M <= 2 (k_row.cu): 16-row x K-slice units
+// taken dynamically, block-diagonal B operand, X converted and kept in
+// shared memory by every CTA.
+struct RowConfig {
+  int M, N, K;
+  int units16, KS, units, IT, ipu, nst, xstride, sp_row, grid;
+  size_t smem, ws_counters_off, ws_gcnt_off, ws_partials_off, ws_bytes;
+};
+cudaError_t row_configure(RowConfig& c, int num_sms);
+// TMA descriptors of one weight set for this variant: one box per unit of 16
+// rows x `ipu` 512-element items (codes with the 128-byte swizzle, scales).
+bool encode_row_maps(int N, int K, int ipu, const uint8_t* wp, const uint8_t* ws, void* map_w,
+                     void* map_s);
+// One launch.
+cudaError_t launch_row(const RowConfig& c, const void* map_w, const void* map_s, const float* gs,
+                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
+                       bool stall, bool pdl, cudaStream_t st);
 
 }  // namespace nvfp4

@@ -13,6 +13,7 @@
 #include <cstdint>
 #include <cuda_fp16.h>
 #include <cuda_bf16.h>
+#include <climits>
 
 namespace nvfp4 {
 
@@ -141,6 +142,21 @@ __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const void* tmap,
       " [%0], [%1, {%2, %3}], [%4], %5;"
       ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(bar), "l"(policy) : "memory");
 }
+// 3D tiled TMA load with an L2 cache policy.
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const void* tmap, int x, int y, int z,
+                                                 uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;"
+      ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy) : "memory");
+}
+// Untiled bulk copy global -> shared (both addresses 16-byte aligned, size a
+// multiple of 16 bytes), completing on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
 __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
@@ -169,6 +185,74 @@ __device__ __forceinline__ int bf16_exp(uint32_t b, uint32_t& sig) {
 __device__ __forceinline__ uint32_t make_f16(uint32_t sign, int t, uint32_t sig) {
   if (t < -14 || t > 15) return 0;
   return (sign << 15) | (uint32_t(t + 15) << 10) | ((sig & 0x7Fu) << 3);
+}
+// f16 bits of sign * sig/128 * 2^t, sig in [128, 255], t <= 15, rounded to
+// nearest even: exact for a normal exponent (t >= -14: 8 significant bits fit
+// the 11 of f16); below that the value is a multiple of the subnormal step
+// 2^-24 after rounding, sig * 2^(t + 17) steps (0 once that is below a half).
+__device__ __forceinline__ uint32_t make_f16_rn(uint32_t sign, int t, uint32_t sig) {
+  if (t >= -14) return make_f16(sign, t, sig);
+  const int sh = t + 17;                       // <= 2
+  uint32_t q;
+  if (sh >= 0) {
+    q = sig << sh;                             // <= 1020: a subnormal mantissa
+  } else {
+    const int n = -sh;
+    if (n > 9) return sign << 15;              // sig / 2^n < 1/2
+    const uint32_t half = 1u << (n - 1), rest = sig & ((1u << n) - 1u);
+    q = sig >> n;
+    if (rest > half || (rest == half && (q & 1u))) ++q;
+  }
+  return (sign << 15) | q;
+}
+
+// Power of two between the hi and the lo f16 plane of X.
+constexpr int X_LO_SHIFT = 29;
+
+// Largest bf16 magnitude (bits, sign cleared) among the eight values of a
+// 16-byte chunk, with one packed 16-bit max per pair.
+__device__ __forceinline__ uint32_t bf16_mag_max8(const uint4& v) {
+  const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
+                              __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+// Exponent floor(log2 |x|) of the bf16 magnitude `mag`; INT_MIN for zero.
+__device__ __forceinline__ int bf16_mag_exp(uint32_t mag) {
+  if (mag == 0u) return INT_MIN;
+  const uint32_t e8 = mag >> 7;
+  if (e8) return int(e8) - 127;
+  return (31 - __clz(int(mag & 0x7Fu))) - 133;     // subnormal
+}
+
+// Two bf16 values (one word) -> their hi f16 pair and lo f16 pair for the
+// token's shift: x * 2^sh (exact: the scale is applied as two powers of two
+// f1 * f2) rounded to f16 is the hi plane (exact for |x * 2^sh| >= 2^-14:
+// 8 significant bits), the exact remainder scaled by 2^X_LO_SHIFT is the lo
+// plane. Returns the lo pair.
+__device__ __forceinline__ uint32_t x_split2(uint32_t w, float f1, float f2, uint32_t& hi) {
+  const float s0 = (__uint_as_float(w << 16) * f1) * f2;
+  const float s1 = (__uint_as_float(w & 0xFFFF0000u) * f1) * f2;
+  const __half2 h = __floats2half2_rn(s0, s1);       // low half = element 0
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  const float2 hb = __half22float2(h);
+  constexpr float kLo = 536870912.0f;                 // 2^X_LO_SHIFT
+  const __half2 l = __floats2half2_rn((s0 - hb.x) * kLo, (s1 - hb.y) * kLo);
+  return *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Eight bf16 values (four words) -> hi and lo planes for the token's shift
+// sh (largest magnitude at 2^14); returns whether any lo element is nonzero.
+__device__ __forceinline__ bool x_split8(const uint32_t w[4], int sh, uint32_t hi[4], uint32_t lo[4]) {
+  static_assert(X_LO_SHIFT == 29, "kLo above is 2^29");
+  const float f1 = __int_as_float((127 + sh / 2) << 23), f2 = __int_as_float((127 + sh - sh / 2) << 23);
+  uint32_t any = 0u;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    lo[q] = x_split2(w[q], f1, f2, hi[q]);
+    any |= lo[q] & 0x7FFF7FFFu;
+  }
+  return any != 0u;
 }
 
 // Number of work-range boundaries floor(c * L / W), c in [1, W), lying in (lo, hi].

@@ -16,8 +16,8 @@ from tests.gpu_util import Guarded, Weights, check_tolerance, dev, host_u16, run
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = [nv.NVFP4_VARIANT_GEMV, nv.NVFP4_VARIANT_MMA, nv.NVFP4_VARIANT_TC]
-VNAME = {0: "auto", 1: "gemv", 2: "mma", 3: "tc"}
+VARIANTS = [nv.NVFP4_VARIANT_GEMV, nv.NVFP4_VARIANT_MMA, nv.NVFP4_VARIANT_TC, nv.NVFP4_VARIANT_ROW]
+VNAME = {0: "auto", 1: "gemv", 2: "mma", 3: "tc", 4: "row"}
 
 _cache = {}
 
@@ -252,8 +252,10 @@ def test_linear_deterministic_and_rows_independent(M):
         assert np.array_equal(y1, y2), VNAME[v]
 
 
-@pytest.mark.parametrize("M", [1, 4, 16])
-def test_pdl_chained_calls_read_the_previous_output(M):
+@pytest.mark.parametrize("variant,M", [(nv.NVFP4_VARIANT_MMA, 1), (nv.NVFP4_VARIANT_MMA, 4),
+                                       (nv.NVFP4_VARIANT_MMA, 16), (nv.NVFP4_VARIANT_ROW, 1),
+                                       (nv.NVFP4_VARIANT_ROW, 2)])
+def test_pdl_chained_calls_read_the_previous_output(variant, M):
     """Programmatic dependent launch: each call's X is the previous call's Y,
     launched back to back on one stream with one shared workspace. Every
     output must match the oracle applied to the GPU's own previous output, so
@@ -267,7 +269,7 @@ def test_pdl_chained_calls_read_the_previous_output(M):
         ws_h.append(oracle.quantize(W))
     dev_w = [Weights(*q) for q in ws_h]
     X0 = synth.x_bf16_custom(synth.X_NORMAL, M, K, seed=9)
-    flags = nv.NVFP4_VARIANT_MMA | nv.NVFP4_PLAN_PDL
+    flags = variant | nv.NVFP4_PLAN_PDL
     plan = nv.nvfp4_linear_plan(M, N, K, torch.cuda.current_device(), flags)
     try:
         wsb = nv.nvfp4_linear_workspace_bytes(plan)
@@ -334,7 +336,8 @@ def test_launches_per_run_counts_the_x_conversion_kernel():
     cases = [(nv.NVFP4_VARIANT_MMA, 1, 1024, 5120, 1), (nv.NVFP4_VARIANT_MMA, 4, 1024, 5120, 1),
              (nv.NVFP4_VARIANT_MMA, 5, 1024, 5120, 2), (nv.NVFP4_VARIANT_MMA, 16, 1024, 5120, 2),
              (nv.NVFP4_VARIANT_TC, 16, 1024, 5120, 1), (nv.NVFP4_VARIANT_GEMV, 1, 1024, 5120, 1),
-             (nv.NVFP4_VARIANT_MMA, 8, 1024, 0, 1), (nv.NVFP4_VARIANT_AUTO, 1, 0, 256, 0)]
+             (nv.NVFP4_VARIANT_MMA, 8, 1024, 0, 1), (nv.NVFP4_VARIANT_AUTO, 1, 0, 256, 0),
+             (nv.NVFP4_VARIANT_ROW, 1, 1024, 5120, 1), (nv.NVFP4_VARIANT_ROW, 2, 1024, 5120, 1)]
     for variant, M, N, K, want in cases:
         plan = nv.nvfp4_linear_plan(M, N, K, d, variant)
         try:
@@ -343,7 +346,7 @@ def test_launches_per_run_counts_the_x_conversion_kernel():
             nv.nvfp4_linear_destroy(plan)
 
 
-@pytest.mark.parametrize("variant", [nv.NVFP4_VARIANT_TC, nv.NVFP4_VARIANT_MMA])
+@pytest.mark.parametrize("variant", [nv.NVFP4_VARIANT_TC, nv.NVFP4_VARIANT_MMA, nv.NVFP4_VARIANT_ROW])
 def test_forced_timeout_reports_status_and_recovers(variant):
     """Test-only flag: the TMA producer never signals, every bounded wait runs
     out, the kernel reports NVFP4_ERR_TIMEOUT through the status word and

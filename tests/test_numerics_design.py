@@ -117,3 +117,34 @@ def test_f16_products_exact_in_f32():
     prod64 = a.astype(np.float64) * b.astype(np.float64)
     prod32 = a.astype(np.float32) * b.astype(np.float32)
     assert np.array_equal(prod32.astype(np.float64), prod64)
+
+
+def _make_f16_rn(sign, t, sig):
+    """The integer rounding of the tcgen05 variant's lo plane, restated: the
+    f16 bits of sign * sig/128 * 2^t (sig in [128, 255]) rounded to nearest
+    even, subnormals included."""
+    if t >= -14:
+        return (sign << 15) | ((t + 15) << 10) | ((sig & 0x7F) << 3)
+    sh = t + 17
+    if sh >= 0:
+        q = sig << sh
+    else:
+        n = -sh
+        if n > 9:
+            return sign << 15
+        half, rest = 1 << (n - 1), sig & ((1 << n) - 1)
+        q = sig >> n
+        if rest > half or (rest == half and (q & 1)):
+            q += 1
+    return (sign << 15) | q
+
+
+def test_integer_f16_rounding_matches_ieee():
+    """Every significand at every exponent from 2^15 down past the last f16
+    subnormal: the integer rounding equals IEEE round-to-nearest-even."""
+    for t in range(-45, 16):
+        for sig in range(128, 256):
+            for sign in (0, 1):
+                v = (-1.0 if sign else 1.0) * sig / 128.0 * 2.0 ** t
+                ref = int(np.array([v], np.float16).view(np.uint16)[0])
+                assert _make_f16_rn(sign, t, sig) == ref, (sign, t, sig)

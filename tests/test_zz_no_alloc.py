@@ -1,7 +1,10 @@
 """nvfp4_linear_run_static: the linear with its split-K scratch in the
 library's fixed device array, checked against nvfp4_linear_run with a caller
-workspace on the same plan. Two calls in a row must both match (the second
-one finds the first one's leftovers in the shared array).
+workspace on the same plan. The reductions are deterministic, so the two
+entry points must agree bit for bit, and both must meet the oracle's
+tolerance. Two calls in a row must both match (the second one finds the
+first one's leftovers in the shared array), also after a run that timed out
+and left its counters behind.
 
 Collected last on purpose: it must pass in a fresh process and after every
 other test has used the device.
@@ -23,6 +26,8 @@ CASES = [
     (nv.NVFP4_VARIANT_TC, 16, 1024, 8192),
     (nv.NVFP4_VARIANT_AUTO, 3, 777, 1280),
     (nv.NVFP4_VARIANT_GEMV, 1, 520, 512),
+    (nv.NVFP4_VARIANT_ROW, 1, 2339, 5120),      # K-split: row-group counters and partials
+    (nv.NVFP4_VARIANT_ROW, 1, 1024, 17408),     # K-split over 17408
 ]
 
 
@@ -36,17 +41,17 @@ def _problem(M, N, K, seed):
 @pytest.mark.parametrize("variant,M,N,K", CASES)
 def test_static_scratch_matches_workspace_entry(variant, M, N, K):
     w, X = _problem(M, N, K, seed=11 + M)
-    _, ad = oracle.linear(w.packed_h, w.scales_h, w.gs, X, M, N, K)
+    y_ref, ad = oracle.linear(w.packed_h, w.scales_h, w.gs, X, M, N, K)
     plan = nv.nvfp4_linear_plan(M, N, K, torch.cuda.current_device(), variant)
     try:
         wsb = nv.nvfp4_linear_workspace_bytes(plan)
         assert wsb <= nv.NVFP4_STATIC_SCRATCH_BYTES
-        if variant in (nv.NVFP4_VARIANT_MMA, nv.NVFP4_VARIANT_TC):
-            # counters and partial sums of split tiles (and X planes for M >= 5)
+        if variant in (nv.NVFP4_VARIANT_MMA, nv.NVFP4_VARIANT_TC, nv.NVFP4_VARIANT_ROW):
+            # counters and partial sums of split tiles (and X planes)
             assert wsb > 256, "case must use the scratch beyond the status word"
         y_ws, ok, _ = run_linear(w, X, plan=plan)
         assert ok
-        y_ref = oracle.bf16_bits_to_f64(y_ws)
+        check_tolerance(y_ws, y_ref, ad)
 
         xd = dev(X)
         stream = torch.cuda.current_stream()
@@ -61,7 +66,43 @@ def test_static_scratch_matches_workspace_entry(variant, M, N, K):
         assert status.tolist() == [0, 0], "device wait status %s" % status.tolist()
         for y in outs:
             assert y.guards_intact()
-            check_tolerance(host_u16(y.view).reshape(M, N), y_ref, ad)
+            got = host_u16(y.view).reshape(M, N)
+            assert (got == y_ws).all(), "static entry differs from the workspace entry"
+            check_tolerance(got, y_ref, ad)
+    finally:
+        nv.nvfp4_linear_destroy(plan)
+
+
+@pytest.mark.parametrize("variant", [nv.NVFP4_VARIANT_MMA, nv.NVFP4_VARIANT_ROW])
+def test_static_scratch_recovers_after_a_timed_out_run(variant):
+    """A test-only plan whose producer never signals runs out its bounded
+    device waits and reports a nonzero status through status_out, leaving
+    counters behind in the shared array; a normal plan of the same shape
+    through the static entry then returns status 0 and the right Y, because
+    every static call clears the counters first."""
+    M, N, K = 1, 2339, 5120
+    w, X = _problem(M, N, K, seed=29)
+    y_ref, ad = oracle.linear(w.packed_h, w.scales_h, w.gs, X, M, N, K)
+    dev_id = torch.cuda.current_device()
+    xd = dev(X)
+    status = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    stalled = nv.nvfp4_linear_plan(M, N, K, dev_id, variant | nv.NVFP4_PLAN_TEST_STALL)
+    try:
+        y = Guarded(M * N)
+        nv.nvfp4_linear_run_static(stalled, w.packed, w.scales, w.gsd, xd, y.view, status[0:1])
+        torch.cuda.synchronize()
+        assert int(status[0].item()) != 0
+        assert y.guards_intact()
+    finally:
+        nv.nvfp4_linear_destroy(stalled)
+    plan = nv.nvfp4_linear_plan(M, N, K, dev_id, variant)
+    try:
+        y = Guarded(M * N)
+        nv.nvfp4_linear_run_static(plan, w.packed, w.scales, w.gsd, xd, y.view, status[1:2])
+        torch.cuda.synchronize()
+        assert int(status[1].item()) == 0
+        assert y.guards_intact()
+        check_tolerance(host_u16(y.view).reshape(M, N), y_ref, ad)
     finally:
         nv.nvfp4_linear_destroy(plan)
 
