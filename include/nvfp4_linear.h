@@ -88,8 +88,29 @@ typedef struct nvfp4_plan_s* nvfp4_plan_t;
 #define NVFP4_VARIANT_ROW  4u  /* M <= 2: 16-row units taken dynamically, warp
                                   MMA with a block-diagonal X operand          */
 #define NVFP4_PLAN_VARIANT_MASK 0xFu
-/* Programmatic dependent launch (MMA and ROW variants; ignored by the others). The
- * launch may start while the previous kernel in the stream is still running:
+/* Fused epilogues (plan flags, bits 8..11; variant MMA, which AUTO takes).
+ * Page "SparkInfer" README, section "Layout & scoring", names fused FFN
+ * kernels; page "Qwen3.8-27B-NVFP4-RTX5090 API & Inference Endpoint",
+ * section "Why lm_head is NVFP4, and why MTP is gone", has the 248,320-row
+ * output projection read for every token, and the greedy decode of page
+ * "SparkInfer" README, section "DSpark speculative decode", needs only each
+ * token's top logit.
+ *   NVFP4_PLAN_EPI_SWIGLU: W is a fused gate+up projection whose rows 2c and
+ *     2c+1 are the gate and up rows of output column c (N even). y is bf16
+ *     [M][N/2]: y[m][c] = silu(g) * u with g, u the complete fp32 values
+ *     gs * acc of rows 2c, 2c+1 and silu(v) = v / (1 + exp(-v)), rounded once
+ *     to bf16.
+ *   NVFP4_PLAN_EPI_ARGMAX: no logits are written. y receives int32 index [M]
+ *     followed by float value [M] (8 M bytes): per token the row n with the
+ *     largest fp32 value gs * acc[n] (not rounded to bf16), equal values
+ *     going to the lower n. The plan's workspace holds the running maxima;
+ *     it is left cleared after the run, like the counters. */
+#define NVFP4_PLAN_EPI_MASK   0xF00u
+#define NVFP4_PLAN_EPI_SWIGLU 0x100u
+#define NVFP4_PLAN_EPI_ARGMAX 0x200u
+/* Programmatic dependent launch (MMA and ROW variants; ignored by the
+ * others). The launch may start while the previous kernel in the stream is
+ * still running:
  * it begins streaming W at once and touches X, Y, w_global and the workspace
  * only after that kernel has completed. So W (codes and scales) must not be
  * written by the kernel launched just before it on the same stream. Back to
@@ -102,10 +123,10 @@ typedef struct nvfp4_plan_s* nvfp4_plan_t;
 
 /* Create a plan for Y[M][N] = X[M][K] W^T on `device`. Chooses the kernel
  * variant (or takes the one forced in `flags`), the split of K and the grid.
- * Returns INVALID_ARG for M outside [1,16], negative N/K, K % 256 != 0 or a
- * null `out`; UNSUPPORTED if a forced variant cannot run this shape; CUDA if
- * the device cannot be queried. On success *out must be released with
- * nvfp4_linear_destroy. */
+ * Returns INVALID_ARG for M outside [1,16], negative N/K, K % 256 != 0, an
+ * unknown epilogue, SWIGLU with N odd, or a null `out`; UNSUPPORTED if a
+ * forced variant cannot run this shape or epilogue; CUDA if the device cannot
+ * be queried. On success *out must be released with nvfp4_linear_destroy. */
 nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
                                nvfp4_plan_t* out);
 
@@ -130,7 +151,8 @@ int nvfp4_linear_launches_per_run(nvfp4_plan_t plan);
 
 /* Run the linear on `stream` (device pointers, see the layout above):
  *   w_packed  uint8 [N][K/2]     w_scales uint8 [N][K/16] (E4M3)
- *   w_global  fp32 [1]           x        bf16 [M][K]       y bf16 [M][N]
+ *   w_global  fp32 [1]           x        bf16 [M][K]
+ *   y         bf16 [M][N], or as the plan's epilogue defines it
  *   workspace >= nvfp4_linear_workspace_bytes(plan) bytes (NULL if 0).
  * Must run on the plan's device (the current device). Returns INVALID_ARG
  * for a null plan or pointer, MISALIGNED for a pointer off its alignment,

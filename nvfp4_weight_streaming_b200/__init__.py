@@ -21,7 +21,7 @@ __all__ = [
     "NVFP4_ERR_CUDA", "NVFP4_ERR_TIMEOUT", "NVFP4_ERR_BAD_SCALE", "NVFP4_ERR_WORKSPACE",
     "NVFP4_VARIANT_AUTO", "NVFP4_VARIANT_GEMV", "NVFP4_VARIANT_MMA", "NVFP4_VARIANT_TC",
     "NVFP4_VARIANT_ROW",
-    "NVFP4_PLAN_PDL", "NVFP4_PLAN_TEST_STALL",
+    "NVFP4_PLAN_PDL", "NVFP4_PLAN_TEST_STALL", "NVFP4_PLAN_EPI_SWIGLU", "NVFP4_PLAN_EPI_ARGMAX",
     "Nvfp4Error", "lib", "library_path",
     "nvfp4_linear_plan", "nvfp4_linear_workspace_bytes", "nvfp4_linear_variant",
     "nvfp4_linear_split_k", "nvfp4_linear_launches_per_run", "nvfp4_linear_run",
@@ -45,6 +45,8 @@ NVFP4_VARIANT_MMA = 2
 NVFP4_VARIANT_TC = 3
 NVFP4_VARIANT_ROW = 4
 NVFP4_PLAN_PDL = 0x10000
+NVFP4_PLAN_EPI_SWIGLU = 0x100
+NVFP4_PLAN_EPI_ARGMAX = 0x200
 NVFP4_PLAN_TEST_STALL = 0x40000000
 NVFP4_STATIC_SCRATCH_BYTES = 16 << 20
 

@@ -31,6 +31,7 @@ struct nvfp4_plan_s {
   int M, N, K, device;
   unsigned flags;
   int variant;
+  int epi;        // fused epilogue: 0 none, 1 SwiGLU, 2 argmax (MMA variant only)
   int split_k;
   int num_sms;
   size_t ws_bytes;
@@ -81,8 +82,8 @@ nvfp4_status static_scratch_address(int device, void** out) {
 // against 105.9 for tcgen05); plan() falls back to tcgen05 for shapes it
 // cannot take.
 int auto_variant(int M, int N, int K) {
-  (void)N; (void)K;
-  return M <= 2 ? int(NVFP4_VARIANT_ROW) : int(NVFP4_VARIANT_MMA);
+  (void)M; (void)N; (void)K;
+  return int(NVFP4_VARIANT_MMA);
 }
 
 // Copy of the TMA descriptors for (wp, ws), encoding them on first use.
@@ -143,6 +144,12 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   if (!out) return NVFP4_ERR_INVALID_ARG;
   *out = nullptr;
   if (M < 1 || M > 16 || N < 0 || K < 0 || K % 256 != 0) return NVFP4_ERR_INVALID_ARG;
+  const unsigned epi_flag = flags & NVFP4_PLAN_EPI_MASK;
+  int epi = 0;
+  if (epi_flag == NVFP4_PLAN_EPI_SWIGLU) epi = 1;
+  else if (epi_flag == NVFP4_PLAN_EPI_ARGMAX) epi = 2;
+  else if (epi_flag != 0u) return NVFP4_ERR_INVALID_ARG;
+  if (epi == 1 && N % 2 != 0) return NVFP4_ERR_INVALID_ARG;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (device < 0 || device >= ndev) return NVFP4_ERR_INVALID_ARG;
@@ -157,6 +164,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   if (!h) { if (prev != device) cudaSetDevice(prev); return NVFP4_ERR_CUDA; }
   nvfp4_plan_s& p = *h;
   p.M = M; p.N = N; p.K = K; p.device = device; p.flags = flags; p.num_sms = sms;
+  p.epi = epi;
   p.split_k = 1;
   p.ws_bytes = 0;
   unsigned forced = flags & NVFP4_PLAN_VARIANT_MASK;
@@ -167,6 +175,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   }
   auto configure = [&]() -> nvfp4_status {
     nvfp4_status st = NVFP4_OK;
+    if (p.epi != 0 && p.variant != int(NVFP4_VARIANT_MMA)) return NVFP4_ERR_UNSUPPORTED;
     switch (p.variant) {
       case NVFP4_VARIANT_GEMV: {
         if (M > 4 || size_t(M) * size_t(K) * 4 > 200 * 1024) { st = NVFP4_ERR_UNSUPPORTED; break; }
@@ -176,7 +185,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
       }
       case NVFP4_VARIANT_MMA: {
         if (K == 0 || N == 0) break;
-        p.mma.M = M; p.mma.N = N; p.mma.K = K;
+        p.mma.M = M; p.mma.N = N; p.mma.K = K; p.mma.epi = p.epi;
         cudaError_t e = nvfp4::mma_configure(p.mma, sms);
         if (e == cudaSuccess && !nvfp4::tensor_maps_supported()) e = cudaErrorNotSupported;
         if (e == cudaErrorInvalidConfiguration || e == cudaErrorNotSupported) st = NVFP4_ERR_UNSUPPORTED;
@@ -219,7 +228,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
     p.ws_bytes = 0;
     st = configure();
   }
-  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.variant != int(NVFP4_VARIANT_TC)) {
+  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.epi == 0 && p.variant != int(NVFP4_VARIANT_TC)) {
     // the automatic choice cannot take this shape: the tcgen05 pipeline can
     p.variant = int(NVFP4_VARIANT_TC);
     p.split_k = 1;
@@ -267,7 +276,9 @@ nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
   const uint16_t* xb = static_cast<const uint16_t*>(x);
   cudaError_t e = cudaSuccess;
   if (K == 0) {
-    e = nvfp4::launch_zero_bf16(yb, int64_t(M) * N, st);
+    // every sum is zero: Y zero, SwiGLU silu(0) * 0 = 0, argmax row 0 with value 0
+    const int64_t count = plan->epi == 1 ? int64_t(M) * (N / 2) : plan->epi == 2 ? 4 * int64_t(M) : int64_t(M) * N;
+    e = nvfp4::launch_zero_bf16(yb, count, st);
   } else {
     switch (plan->variant) {
       case NVFP4_VARIANT_GEMV:

@@ -103,9 +103,106 @@ struct Params {
   uint32_t* status;
   uint32_t* counters;
   float* partials;
+  unsigned long long* keys;                  // argmax epilogue: per-token best (value, index) key
+  uint32_t* done;                            // argmax epilogue: CTAs finished
   long long timeout;
   int stall;
 };
+
+// ---- epilogues --------------------------------------------------------------
+// EPI_NONE: y[m][n] = bf16(gs * acc). EPI_SWIGLU (fused gate+up projection,
+// rows 2c and 2c+1 are the gate and up rows of output column c): y[m][c] =
+// bf16(silu(gs * acc_2c) * gs * acc_2c+1), computed in fp32 from the complete
+// sums. EPI_ARGMAX (greedy choice over the output vocabulary): per token the
+// largest fp32 logit gs * acc and its row, equal values going to the lower
+// row; no logits are written. The candidates meet as 64-bit keys (order-
+// preserving bits of the value above the complemented row index) in one
+// atomic maximum per token and warp; the last CTA to finish writes
+// int32 index [M] then float value [M] to y and clears the keys.
+constexpr int EPI_NONE = 0, EPI_SWIGLU = 1, EPI_ARGMAX = 2;
+
+__device__ __forceinline__ float silu(float v) { return v / (1.0f + expf(-v)); }
+
+__device__ __forceinline__ unsigned long long argmax_key(float v, int n) {
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return (static_cast<unsigned long long>(ord) << 32) | (0xFFFFFFFFu - uint32_t(n));
+}
+__device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned mask, unsigned long long v, int o) {
+  const uint32_t lo = __shfl_xor_sync(mask, uint32_t(v), o), hi = __shfl_xor_sync(mask, uint32_t(v >> 32), o);
+  return (static_cast<unsigned long long>(hi) << 32) | lo;
+}
+
+// Token of accumulator value e of a lane in quad position t, or -1: the
+// columns 2t, 2t+1 of the first token tile (e = 0, 1) and of the second
+// (e = 2, 3; M > 8).
+template <int MC>
+__device__ __forceinline__ int tok_of(int t, int e) {
+  if (MC == 1) return (t < 2 && e < 2) ? 2 * t + e : -1;
+  if (e < 2) return 2 * t + e;
+  return MC == 3 ? 8 + 2 * t + (e - 2) : -1;
+}
+
+// Complete sums (before the global scale) of a lane's rows row0 and row0 + 8
+// for its tokens, stored as the plan's epilogue asks. All 32 lanes of the
+// warp call it together (the epilogues exchange values across lanes).
+template <int MC, int EPI>
+__device__ __forceinline__ void emit_rows(const Params& p, int row0, const float (&val)[4][2], float gs,
+                                          int lane) {
+  const int t = lane & 3, g = lane >> 2;
+  if constexpr (EPI == EPI_NONE) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int m = tok_of<MC>(t, e);
+      if (m >= 0 && m < p.M) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int n = row0 + 8 * h;
+          if (n < p.N) p.y[size_t(m) * p.N + n] = float_to_bf16_bits(gs * val[e][h]);
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    // rows row0 and row0 + 8 pair with the rows of the lane g ^ 1
+    float up[4][2];
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) up[e][h] = __shfl_xor_sync(0xffffffffu, val[e][h], 4);
+    if ((g & 1) == 0) {
+      const int half = p.N >> 1;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int m = tok_of<MC>(t, e);
+        if (m >= 0 && m < p.M) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int n = row0 + 8 * h;
+            if (n < p.N) p.y[size_t(m) * half + (n >> 1)] = float_to_bf16_bits(silu(gs * val[e][h]) * (gs * up[e][h]));
+          }
+        }
+      }
+    }
+  } else {
+    // the eight lanes g = 0..7 of a quad position hold the same tokens
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int m = tok_of<MC>(t, e);
+      unsigned long long key = 0ull;
+      if (m >= 0 && m < p.M) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int n = row0 + 8 * h;
+          if (n < p.N) key = max(key, argmax_key(gs * val[e][h], n));
+        }
+      }
+      key = max(key, shfl_xor_u64(0xffffffffu, key, 4));
+      key = max(key, shfl_xor_u64(0xffffffffu, key, 8));
+      key = max(key, shfl_xor_u64(0xffffffffu, key, 16));
+      if (g == 0 && m >= 0 && m < p.M) atomicMax(p.keys + m, key);
+    }
+  }
+}
 
 // Byte offset of X element k (local to the slice) inside a column: groups of
 // 64 elements take 136 bytes (8 bytes of padding), so the four lanes t of an
@@ -194,6 +291,7 @@ __device__ __forceinline__ int list_pieces(const Params& p, int tile, uint32_t* 
 
 // Y rows of the row groups in `gmask` of `tile` = sum of all pieces in k
 // order (first piece first), for threads tid, tid + nth, ...
+template <int EPI>
 __device__ __forceinline__ void sum_pieces(const Params& p, int tile, uint32_t gmask,
                                            const uint32_t* pieces, int np, int tid, int nth) {
   const float gs = *p.gs;
@@ -214,7 +312,22 @@ __device__ __forceinline__ void sum_pieces(const Params& p, int tile, uint32_t g
     }
     for (; o < np; ++o) sum += __ldcg(base + size_t(pieces[o]) * MT);
     const int n = tile * TROWS + row;
-    if (n < p.N) p.y[size_t(m) * p.N + n] = float_to_bf16_bits(gs * sum);
+    if constexpr (EPI == EPI_NONE) {
+      if (n < p.N) p.y[size_t(m) * p.N + n] = float_to_bf16_bits(gs * sum);
+    } else if constexpr (EPI == EPI_SWIGLU) {
+      // consecutive u are consecutive rows of one token: the partner is u ^ 1
+      const float up = __shfl_xor_sync(__activemask(), sum, 1);
+      if ((rr & 1) == 0 && n < p.N) p.y[size_t(m) * (p.N >> 1) + (n >> 1)] = float_to_bf16_bits(silu(gs * sum) * (gs * up));
+    } else {
+      // the 16 consecutive u of a row group share the token
+      const unsigned mask = __activemask();
+      unsigned long long key = n < p.N ? argmax_key(gs * sum, n) : 0ull;
+      key = max(key, shfl_xor_u64(mask, key, 1));
+      key = max(key, shfl_xor_u64(mask, key, 2));
+      key = max(key, shfl_xor_u64(mask, key, 4));
+      key = max(key, shfl_xor_u64(mask, key, 8));
+      if (rr == 0) atomicMax(p.keys + m, key);
+    }
   }
 }
 
@@ -335,7 +448,7 @@ __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* s
 // one tile; 2: hi + lo tiles, or two hi tiles; 4: two hi + two lo tiles).
 // Pieces of split tiles are written to the workspace and handed to the
 // settler warp through the queue (mbarriers q_full / q_empty).
-template <int MC, int NTILE, bool LO, bool XR>
+template <int MC, int NTILE, bool LO, bool XR, int EPI>
 __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* sS, const uint8_t* sX,
                                         const int* emax, uint32_t b_full, uint32_t b_empty,
                                         uint32_t b_qfull, uint32_t b_qempty,
@@ -346,11 +459,7 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
   const int r = 16 * cw + g;                           // row of the tile (and r + 8)
   // tokens of this lane's accumulator values (columns 2t, 2t+1 of a tile):
   // e = 0, 1 from the first token tile, e = 2, 3 from the second (M > 8)
-  auto tok = [t](int e) {
-    if (MC == 1) return (t < 2 && e < 2) ? 2 * t + e : -1;
-    if (e < 2) return 2 * t + e;
-    return MC == 3 ? 8 + 2 * t + (e - 2) : -1;
-  };
+  auto tok = [t](int e) { return tok_of<MC>(t, e); };
   // X column of each token tile for this lane (B column g); shared memory
   // holds only the 2M used columns: hi plane tokens 0..M-1, then lo plane.
   // LO: some lo element is nonzero, lanes of absent tokens skip their loads
@@ -468,16 +577,9 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     const int this_start = seg_start;
     seg_start = idx + 1;
     const bool whole = (p.S == 1) && (this_start == tcur * cnt) && (jcur + 1 == cnt);
-    const int row0 = tcur * TROWS + r, row1 = row0 + 8;
+    const int row0 = tcur * TROWS + r;
     if (whole) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int m = tok(e);
-        if (m >= 0 && m < p.M) {
-          if (row0 < p.N) p.y[size_t(m) * p.N + row0] = float_to_bf16_bits(gs * v[e][0]);
-          if (row1 < p.N) p.y[size_t(m) * p.N + row1] = float_to_bf16_bits(gs * v[e][1]);
-        }
-      }
+      emit_rows<MC, EPI>(p, row0, v, gs, lane);
       continue;
     }
     // piece of a split tile
@@ -493,14 +595,15 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
         __all_sync(0xffffffffu, *pre_flag != 0u)) {
       // the settler has copied the other piece into shared memory
       __threadfence_block();
+      float sum[4][2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
+      for (int e = 0; e < 4; ++e) {
         const int m = tok(e);
-        if (m >= 0 && m < p.M) {
-          if (row0 < p.N) p.y[size_t(m) * p.N + row0] = float_to_bf16_bits(gs * (v[e][0] + pre_buf[m * TROWS + r]));
-          if (row1 < p.N) p.y[size_t(m) * p.N + row1] = float_to_bf16_bits(gs * (v[e][1] + pre_buf[m * TROWS + r + 8]));
-        }
+        const bool ok_m = m >= 0 && m < p.M;
+        sum[e][0] = v[e][0] + (ok_m ? pre_buf[m * TROWS + r] : 0.0f);
+        sum[e][1] = v[e][1] + (ok_m ? pre_buf[m * TROWS + r + 8] : 0.0f);
       }
+      emit_rows<MC, EPI>(p, row0, sum, gs, lane);
       __syncwarp();
       if (lane == 0) *reinterpret_cast<volatile uint32_t*>(p.counters + tcur * NCW + cw) = 0u;
       done_here = true;
@@ -532,14 +635,7 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
               }
             }
           }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int m = tok(e);
-            if (m >= 0 && m < p.M) {
-              if (row0 < p.N) p.y[size_t(m) * p.N + row0] = float_to_bf16_bits(gs * sum[e][0]);
-              if (row1 < p.N) p.y[size_t(m) * p.N + row1] = float_to_bf16_bits(gs * sum[e][1]);
-            }
-          }
+          emit_rows<MC, EPI>(p, row0, sum, gs, lane);
           __syncwarp();
           if (lane == 0) *reinterpret_cast<volatile uint32_t*>(ctr) = 0u;
           done_here = true;
@@ -575,6 +671,7 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
 // this CTA brought the last piece are listed for the end phase, where all
 // warps of the CTA add the pieces; if the list is full the settler adds them
 // itself.
+template <int EPI>
 __device__ __forceinline__ void settle(const Params& p, uint32_t b_qfull, uint32_t b_qempty,
                                        volatile int* abort_flag, uint32_t* skip, uint32_t* list,
                                        uint32_t* nlist, uint32_t* pieces, volatile uint32_t* pre_flag,
@@ -644,7 +741,7 @@ __device__ __forceinline__ void settle(const Params& p, uint32_t b_qfull, uint32
         if (lane == 0) pieces[MAX_PIECES] = uint32_t(list_pieces(p, tcur, pieces));
         __syncwarp();
         __threadfence();
-        sum_pieces(p, tcur, lastmask, pieces, int(pieces[MAX_PIECES]), lane, 32);
+        sum_pieces<EPI>(p, tcur, lastmask, pieces, int(pieces[MAX_PIECES]), lane, 32);
         if ((lastmask >> lane) & 1u) p.counters[tcur * NCW + lane] = 0u;
       }
     }
@@ -660,7 +757,7 @@ __device__ __forceinline__ void settle(const Params& p, uint32_t b_qfull, uint32
 // XR: X in the ring. Each stage also carries one K-step of the X planes
 // (prepared by k_xprep in the workspace), there are no K-slices and no
 // staging; otherwise the CTA stages its K-slice of X in shared memory.
-template <int MC, bool XR>
+template <int MC, bool XR, int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
       const __grid_constant__ CUtensorMap tm_x, const Params p) {
@@ -765,14 +862,14 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
   } else if (warp == WARP_SETTLE) {
     // ---------------------------------------------------------------- settler
     asm volatile("griddepcontrol.wait;" ::: "memory");   // counters of the previous grid
-    settle(p, b_qfull, b_qempty, abort_flag, skip, list, flags + 2, pieces, pre_flag, pre_buf, cnt, a, b, L, lane);
+    settle<EPI>(p, b_qfull, b_qempty, abort_flag, skip, list, flags + 2, pieces, pre_flag, pre_buf, cnt, a, b, L, lane);
   } else {
     // ------------------------------------------------ consumers: stage X first
     // X, the global scale, Y and the workspace may belong to the previous grid
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int cw = warp - 1;
 #define NVFP4_CONSUME(MC_, NT_, LO_, XR_, EMAX_) \
-  consume<MC_, NT_, LO_, XR_>(p, sW, sS, sX, EMAX_, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, pre_flag, pre_buf, s, cnt, a, b, L, cw, lane)
+  consume<MC_, NT_, LO_, XR_, EPI>(p, sW, sS, sX, EMAX_, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, pre_flag, pre_buf, s, cnt, a, b, L, cw, lane)
     if constexpr (XR) {
       // X arrives with the weights; exponents and lo flags come from k_xprep
       bool need_lo = false;
@@ -862,18 +959,63 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
       const uint32_t gmask = list[2 * e + 1];
       if (threadIdx.x == 0) pieces[MAX_PIECES] = uint32_t(list_pieces(p, tile, pieces));
       __syncthreads();
-      sum_pieces(p, tile, gmask, pieces, int(pieces[MAX_PIECES]), threadIdx.x, NUM_THREADS);
+      sum_pieces<EPI>(p, tile, gmask, pieces, int(pieces[MAX_PIECES]), threadIdx.x, NUM_THREADS);
       if (threadIdx.x < NCW && ((gmask >> threadIdx.x) & 1u)) p.counters[tile * NCW + threadIdx.x] = 0u;
       __syncthreads();
+    }
+  }
+  if constexpr (EPI == EPI_ARGMAX) {
+    // the last CTA to finish turns the per-token keys into (index, value)
+    __syncthreads();
+    if (threadIdx.x == 0 && !*abort_flag) {
+      __threadfence();
+      if (atomicAdd(p.done, 1u) == gridDim.x - 1) {
+        __threadfence();
+        int* out_idx = reinterpret_cast<int*>(p.y);
+        float* out_val = reinterpret_cast<float*>(out_idx + p.M);
+        for (int m = 0; m < p.M; ++m) {
+          const unsigned long long key = atomicExch(p.keys + m, 0ull);
+          const uint32_t ord = uint32_t(key >> 32);
+          out_idx[m] = int(0xFFFFFFFFu - uint32_t(key));
+          out_val[m] = __uint_as_float((ord & 0x80000000u) ? (ord & 0x7FFFFFFFu) : ~ord);
+        }
+        *p.done = 0u;
+      }
     }
   }
 }
 
 }  // namespace mm
 
+// The kernels' opt-in shared memory (every instantiation the launcher uses).
+template <int EPI>
+cudaError_t set_smem_attrs(int optin) {
+  using namespace mm;
+  cudaError_t e = cudaFuncSetAttribute(k_mma<1, false, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<1, true, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<2, true, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<3, true, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  return e;
+}
+
+// Launch of the main kernel for one epilogue.
+template <int EPI>
+cudaError_t launch_main(const MmaConfig& c, cudaLaunchConfig_t* cfg, const CUtensorMap& mw, const CUtensorMap& ms,
+                        const CUtensorMap& mx, const mm::Params& p) {
+  using namespace mm;
+  if (c.M <= 4) {
+    if (c.xr) return cudaLaunchKernelEx(cfg, k_mma<1, true, EPI>, mw, ms, mx, p);
+    return cudaLaunchKernelEx(cfg, k_mma<1, false, EPI>, mw, ms, mx, p);
+  }
+  if (c.M <= 8) return cudaLaunchKernelEx(cfg, k_mma<2, true, EPI>, mw, ms, mx, p);
+  return cudaLaunchKernelEx(cfg, k_mma<3, true, EPI>, mw, ms, mx, p);
+}
+
 cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   using namespace mm;
   if (c.M < 1 || c.M > 16 || c.K % KS != 0 || c.K <= 0 || c.N <= 0) return cudaErrorInvalidValue;
+  if (c.epi < EPI_NONE || c.epi > EPI_ARGMAX || (c.epi == EPI_SWIGLU && c.N % 2 != 0))
+    return cudaErrorInvalidConfiguration;
   int dev = 0, optin = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -945,9 +1087,11 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   // workspace: status word, per-(tile, row group) counters, partial sums,
   // and for X in the ring the X planes plus per-token exponent and lo flag
   c.ws_counters_off = 256;
-  c.ws_partials_off = c.ws_counters_off + ((size_t(c.tiles) * NCW * 4 + 255) / 256) * 256;
+  // argmax epilogue state (per-token keys, finished-CTA counter) after the counters
+  c.ws_epi_off = c.ws_counters_off + ((size_t(c.tiles) * NCW * 4 + 255) / 256) * 256;
+  c.ws_partials_off = c.ws_epi_off + 256;
   const size_t partials_end = split ? c.ws_partials_off + size_t(c.tiles) * S * pmax * c.M * TROWS * 4
-                                    : (c.xr ? c.ws_partials_off : 256);
+                                    : ((c.xr || c.epi == EPI_ARGMAX) ? c.ws_partials_off : 256);
   if (c.xr) {
     c.ws_x_off = ((partials_end + 255) / 256) * 256;
     c.ws_xmeta_off = c.ws_x_off + ((size_t(c.ncols) * c.x_pitch + 255) / 256) * 256;
@@ -956,10 +1100,9 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
     c.ws_x_off = c.ws_xmeta_off = 0;
     c.ws_bytes = partials_end;
   }
-  e = cudaFuncSetAttribute(k_mma<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  e = set_smem_attrs<EPI_NONE>(optin);
+  if (e == cudaSuccess) e = set_smem_attrs<EPI_SWIGLU>(optin);
+  if (e == cudaSuccess) e = set_smem_attrs<EPI_ARGMAX>(optin);
   return e;
 }
 
@@ -979,6 +1122,8 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
   p.partials = c.split ? reinterpret_cast<float*>(wsb + c.ws_partials_off) : nullptr;
   p.xemax = c.xr ? reinterpret_cast<const int*>(wsb + c.ws_xmeta_off) : nullptr;
   p.xlo = c.xr ? reinterpret_cast<const uint32_t*>(wsb + c.ws_xmeta_off + 64) : nullptr;
+  p.keys = reinterpret_cast<unsigned long long*>(wsb + c.ws_epi_off);
+  p.done = reinterpret_cast<uint32_t*>(wsb + c.ws_epi_off + 128);
   p.timeout = timeout_cycles;
   p.stall = stall ? 1 : 0;
   const CUtensorMap& mw = *static_cast<const CUtensorMap*>(map_w);
@@ -1007,12 +1152,9 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
   cfg.attrs = attr;
   // after k_xprep the dependency is always programmatic: k_mma waits for it in-kernel
   cfg.numAttrs = (pdl || c.xr) ? 1 : 0;
-  if (c.M <= 4) {
-    if (c.xr) return cudaLaunchKernelEx(&cfg, k_mma<1, true>, mw, ms, mx, p);
-    return cudaLaunchKernelEx(&cfg, k_mma<1, false>, mw, ms, mx, p);
-  }
-  if (c.M <= 8) return cudaLaunchKernelEx(&cfg, k_mma<2, true>, mw, ms, mx, p);
-  return cudaLaunchKernelEx(&cfg, k_mma<3, true>, mw, ms, mx, p);
+  if (c.epi == EPI_SWIGLU) return launch_main<EPI_SWIGLU>(c, &cfg, mw, ms, mx, p);
+  if (c.epi == EPI_ARGMAX) return launch_main<EPI_ARGMAX>(c, &cfg, mw, ms, mx, p);
+  return launch_main<EPI_NONE>(c, &cfg, mw, ms, mx, p);
 }
 
 }  // namespace nvfp4

@@ -55,13 +55,14 @@ cudaError_t launch_tc(const TcConfig& c, const void* map_w, const void* map_s, c
 // Register-direct warp-MMA variant (k_mma.cu).
 struct MmaConfig {
   int M, N, K;
+  int epi;   // 0: Y; 1: SiLU-gated pairs of rows; 2: per-token argmax (k_mma.cu)
   int tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, nstage, grid;
   bool split;
   // X in the ring (M > 4): X planes prepared once per call in the workspace
   bool xr;
   int x_pitch, x_box, xbytes;
   size_t ws_x_off, ws_xmeta_off;
-  size_t smem, ws_counters_off, ws_partials_off, ws_bytes;
+  size_t smem, ws_counters_off, ws_epi_off, ws_partials_off, ws_bytes;
 };
 cudaError_t mma_configure(MmaConfig& c, int num_sms);
 // map_x: descriptor of the X planes in `workspace` (encode_x_planes_map), used when c.xr.
