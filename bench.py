@@ -36,8 +36,13 @@ VARIANT_NAMES = ("auto", "gemv", "mma", "tc", "row")
 FALLBACK_HBM_GBS = 6650.0
 
 
-def bytes_per_call(M: int, N: int, K: int) -> int:
-    return N * K // 2 + N * K // 16 + 2 * M * K + 2 * M * N
+def bytes_per_call(M: int, N: int, K: int, fmt: str = "nvfp4", epi: str = "none") -> int:
+    """Algorithmic bytes of one call: weights (NVFP4 codes and E4M3 scales, or
+    FP8 codes and fp32 row scales), X, and the output (Y; N/2 columns with the
+    SwiGLU epilogue; an int32 index and a float value per token with argmax)."""
+    wbytes = N * K // 2 + N * K // 16 if fmt == "nvfp4" else N * K + 4 * N
+    out = {"none": 2 * M * N, "swiglu": M * N, "argmax": 8 * M}[epi]
+    return wbytes + 2 * M * K + out
 
 
 def effective_gbs(nbytes: float, seconds: float) -> float:
@@ -172,9 +177,12 @@ def aggregate(world: int, bytes_per_call: float, sec_per_call_this_rank: float):
 # ---------------------------------------------------------------------------
 
 class Problem:
-    """One workload on the device: weight copies, X, Y, plan, workspace."""
+    """One workload on the device: weight copies, X, Y, plan, workspace.
+    fmt "nvfp4" (the method) or "fp8" (the comparison tier); epi "none",
+    "swiglu" or "argmax" (fused epilogues)."""
 
-    def __init__(self, name: str, M: int, variant: int, min_footprint: float, flags: int = 0):
+    def __init__(self, name: str, M: int, variant: int, min_footprint: float, flags: int = 0,
+                 fmt: str = "nvfp4", epi: str = "none"):
         import numpy as np
         import torch
         import synth
@@ -183,17 +191,26 @@ class Problem:
         wl = synth.WORKLOADS[name]
         self.name, self.M, self.N, self.K = name, M, wl.N, wl.K
         dev = torch.cuda.current_device()
+        self.fmt, self.epi = fmt, epi
         # weights: generated on the host, quantised on the device by the library
         W = torch.from_numpy(synth.weights_f32(wl)).cuda()
-        packed = torch.empty((self.N, self.K // 2), dtype=torch.uint8, device="cuda")
-        scales = torch.empty((self.N, self.K // 16), dtype=torch.uint8, device="cuda")
-        gs = torch.empty(1, dtype=torch.float32, device="cuda")
         bad = torch.zeros(1, dtype=torch.int32, device="cuda")
-        nv.nvfp4_quantize(W, self.N, self.K, packed, scales, gs, bad)
+        if fmt == "nvfp4":
+            packed = torch.empty((self.N, self.K // 2), dtype=torch.uint8, device="cuda")
+            scales = torch.empty((self.N, self.K // 16), dtype=torch.uint8, device="cuda")
+            gs = torch.empty(1, dtype=torch.float32, device="cuda")
+            nv.nvfp4_quantize(W, self.N, self.K, packed, scales, gs, bad)
+        else:
+            packed = torch.empty((self.N, self.K), dtype=torch.uint8, device="cuda")
+            scales = torch.empty(self.N, dtype=torch.float32, device="cuda")
+            gs = torch.ones(1, dtype=torch.float32, device="cuda")
+            nv.nvfp4_quantize_fp8(W, self.N, self.K, packed, scales, bad)
+            flags |= nv.NVFP4_PLAN_WEIGHT_FP8
+        flags |= {"none": 0, "swiglu": nv.NVFP4_PLAN_EPI_SWIGLU, "argmax": nv.NVFP4_PLAN_EPI_ARGMAX}[epi]
         torch.cuda.synchronize()
         assert int(bad.item()) == 0
         del W
-        wbytes = packed.numel() + scales.numel()
+        wbytes = packed.numel() * packed.element_size() + scales.numel() * scales.element_size()
         self.ncopies = max(1, math.ceil(min_footprint / wbytes))
         self.copies = [(packed, scales)] + [(packed.clone(), scales.clone())
                                             for _ in range(self.ncopies - 1)]
@@ -201,14 +218,15 @@ class Problem:
         xh = synth.x_bf16(wl, M)
         self.x_host = xh
         self.x = torch.from_numpy(xh.view(np.int16)).cuda()
-        self.y = torch.empty((M, self.N), dtype=torch.int16, device="cuda")
+        ycount = {"none": M * self.N, "swiglu": M * (self.N // 2), "argmax": 4 * M}[epi]
+        self.y = torch.empty(ycount, dtype=torch.int16, device="cuda")
         self.plan = nv.nvfp4_linear_plan(M, self.N, self.K, dev, variant | flags)
         self.flags = flags
         self.variant = nv.nvfp4_linear_variant(self.plan)
         self.split_k = nv.nvfp4_linear_split_k(self.plan)
         self.wsb = nv.nvfp4_linear_workspace_bytes(self.plan)
         self.ws = torch.zeros(max(self.wsb, 16), dtype=torch.uint8, device="cuda")
-        self.bytes = bytes_per_call(M, self.N, self.K)
+        self.bytes = bytes_per_call(M, self.N, self.K, fmt, epi)
         self.footprint = wbytes * self.ncopies
         self.lib = nv.lib()
 
@@ -233,10 +251,12 @@ class Problem:
 
 
 def time_problem(pb: Problem, steps: int, warmup: int, world: int, graph_len: int = 64,
-                 sampler: ClockSampler | None = None):
+                 sampler: ClockSampler | None = None, repeats: int = 1):
     """Warm up, then time exactly `steps` calls (replayed from CUDA graphs of
-    `graph_len` calls) between CUDA events; returns seconds per call (max over
-    ranks) and the number of kernel launches timed."""
+    `graph_len` calls) between CUDA events, `repeats` times; returns the
+    median seconds per call (each repeat's time is the max over ranks), the
+    number of kernel launches in one timed block, and every repeat's seconds
+    per call."""
     import torch
     stream = torch.cuda.Stream()
     torch.cuda.synchronize()
@@ -266,26 +286,29 @@ def time_problem(pb: Problem, steps: int, warmup: int, world: int, graph_len: in
     stream.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize()
-    if sampler:
-        sampler.mark("t0")
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(steps // glen):
-            graph.replay()
-        if tail_graph is not None:
-            tail_graph.replay()
-        e1.record(stream)
-    stream.synchronize()
-    torch.cuda.synchronize()
+    per_call = []
+    for rep in range(max(1, repeats)):
+        barrier(world)
+        torch.cuda.synchronize()
+        if sampler and rep == 0:
+            sampler.mark("t0")
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps // glen):
+                graph.replay()
+            if tail_graph is not None:
+                tail_graph.replay()
+            e1.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize()
+        barrier(world)
+        per_call.append(max_over_ranks(world, e0.elapsed_time(e1) / 1e3) / steps)
     if sampler:
         sampler.mark("t1")
-    barrier(world)
-    sec = e0.elapsed_time(e1) / 1e3
     pb.check_status()
     del graph, tail_graph
-    return max_over_ranks(world, sec) / steps, steps * pb.nv.nvfp4_linear_launches_per_run(pb.plan)
+    return (statistics.median(per_call), steps * pb.nv.nvfp4_linear_launches_per_run(pb.plan),
+            per_call)
 
 
 def time_e2e(pb: Problem, steps: int, world: int):
@@ -398,23 +421,38 @@ def run_ours(args):
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if sampler:
         sampler.start()
-    sec, launches = time_problem(pb, args.steps, args.warmup, world, sampler=sampler)
+    sec, launches, reps = time_problem(pb, args.steps, args.warmup, world, sampler=sampler,
+                                       repeats=args.repeats)
     clocks = sampler.stop() if sampler else None
     value = effective_gbs(pb.bytes * world, sec)
     per_gpu = effective_gbs(pb.bytes, sec)
     sweep = []
     if not args.no_sweep:
-        for (name, M) in ([("verify", 16)] if not args.full_sweep else
-                          [("verify", m) for m in (1, 2, 4, 8, 12, 16)] +
-                          [("down", m) for m in (1, 4, 8, 16)] +
-                          [("lm_head", m) for m in (1, 8, 16)]):
-            q = Problem(name, M, variant, min_footprint=4.2 * l2, flags=flags)
-            s2, _ = time_problem(q, max(args.steps, 200), args.warmup, world)
+        # every workload shape and M (the down projection's 64 rotated copies
+        # included), then the fused epilogues and the FP8 comparison tier
+        points = [("verify", m, "nvfp4", "none") for m in (1, 2, 4, 8, 12, 16)] + \
+                 [("down", m, "nvfp4", "none") for m in (1, 4, 8, 16)] + \
+                 [("lm_head", m, "nvfp4", "none") for m in (1, 8, 16)] + \
+                 [("verify", m, "nvfp4", "swiglu") for m in (1, 16)] + \
+                 [("lm_head", m, "nvfp4", "argmax") for m in (1, 16)] + \
+                 [("verify", m, "fp8", "none") for m in (1, 2)] + \
+                 [("down", 1, "fp8", "none"), ("lm_head", 1, "fp8", "none")]
+        base_us = {}
+        for (name, M, fmt, epi) in points:
+            v = variant if (fmt == "nvfp4" and epi == "none") else 0
+            q = Problem(name, M, v, min_footprint=4.2 * l2, flags=flags, fmt=fmt, epi=epi)
+            s2, _, r2 = time_problem(q, max(args.steps, 200), args.warmup, world, repeats=args.repeats)
             g = effective_gbs(q.bytes, s2)
-            sweep.append({"workload": name, "M": M, "N": q.N, "K": q.K,
-                          "variant": VARIANT_NAMES[q.variant],
-                          "split_k": q.split_k, "us_per_call": s2 * 1e6, "GBps": g,
-                          "frac_of_measured_peak": g / peak})
+            pt = {"workload": name, "M": M, "N": q.N, "K": q.K, "weights": fmt, "epilogue": epi,
+                  "variant": VARIANT_NAMES[q.variant], "split_k": q.split_k,
+                  "bytes_per_call": q.bytes, "us_per_call": s2 * 1e6,
+                  "us_spread": [min(r2) * 1e6, max(r2) * 1e6], "GBps": g,
+                  "frac_of_measured_peak": g / peak}
+            if fmt == "nvfp4" and epi == "none":
+                base_us[(name, M)] = s2 * 1e6
+            elif (name, M) in base_us:
+                pt["time_over_plain_nvfp4"] = s2 * 1e6 / base_us[(name, M)]
+            sweep.append(pt)
             q.destroy()
             del q
             torch.cuda.empty_cache()
@@ -430,6 +468,7 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+            "repeats": len(reps), "ms_per_step_spread": [min(reps) * 1e3, max(reps) * 1e3],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "nvfp4 weights x bf16 activations, f16 products, f32 accumulate",
             "data": "synthetic (seeded SplitMix64/Box-Muller, workload recipes in synth/)",
@@ -543,7 +582,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch")
-    ap.add_argument("--full-sweep", action="store_true")
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="timed blocks of --steps calls; the median is reported")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-rows", type=int, default=0,

@@ -105,6 +105,17 @@ typedef struct nvfp4_plan_s* nvfp4_plan_t;
  *     largest fp32 value gs * acc[n] (not rounded to bf16), equal values
  *     going to the lower n. The plan's workspace holds the running maxima;
  *     it is left cleared after the run, like the counters. */
+/* FP8 weight tier (plan flag; variant ROW, so M <= 2): W is stored as E4M3
+ * codes, one byte per element, with one fp32 scale per row, for comparison
+ * with NVFP4 at the same shapes (page "Qwen3.8-27B-NVFP4-RTX5090 API &
+ * Inference Endpoint", section "Measured against the other NVFP4 builds of
+ * this model": the next instruction tier costs 1.5-2.1x on these GEMM
+ * shapes; page "InventDB Sparkle", section "How it answers quickly": 8-bit
+ * weights). With this flag w_packed is uint8 [N][K] (E4M3 codes), w_scales
+ * is float [N] and w_hat[n][k] = e4m3(code[n][k]) * w_scales[n] * gs; X, Y,
+ * the tolerance and the X range are as for NVFP4. nvfp4_quantize_fp8 makes
+ * such weights. */
+#define NVFP4_PLAN_WEIGHT_FP8 0x1000u
 #define NVFP4_PLAN_EPI_MASK   0xF00u
 #define NVFP4_PLAN_EPI_SWIGLU 0x100u
 #define NVFP4_PLAN_EPI_ARGMAX 0x200u
@@ -228,6 +239,16 @@ nvfp4_status nvfp4_pack_check(const uint8_t* w_packed, const uint8_t* w_scales,
 nvfp4_status nvfp4_quantize(const float* w, int N, int K, uint8_t* w_packed,
                             uint8_t* w_scales, float* w_global, unsigned* d_bad,
                             void* stream);
+
+/* FP8 weight tier quantiser: fp32 W [N][K] (device) -> E4M3 codes uint8
+ * [N][K] and fp32 row scales [N]: s_n = amax |W[n]| / 448, code =
+ * E4M3_RNE_satfinite(w / s_n), each step one fp32 operation; a row with
+ * s_n = 0 gets all-zero codes, and a negative value that rounds to zero keeps
+ * its sign (0x80). *d_bad (nullable, caller-zeroed) receives the number of
+ * non-finite elements (the outputs are then unspecified). K % 16 == 0;
+ * pointers 16-byte aligned. One kernel on `stream`. */
+nvfp4_status nvfp4_quantize_fp8(const float* w, int N, int K, uint8_t* codes, float* row_scales,
+                                unsigned* d_bad, void* stream);
 
 /* Static text for a status code. */
 const char* nvfp4_status_string(nvfp4_status s);

@@ -22,6 +22,7 @@ __all__ = [
     "NVFP4_VARIANT_AUTO", "NVFP4_VARIANT_GEMV", "NVFP4_VARIANT_MMA", "NVFP4_VARIANT_TC",
     "NVFP4_VARIANT_ROW",
     "NVFP4_PLAN_PDL", "NVFP4_PLAN_TEST_STALL", "NVFP4_PLAN_EPI_SWIGLU", "NVFP4_PLAN_EPI_ARGMAX",
+    "NVFP4_PLAN_WEIGHT_FP8", "nvfp4_quantize_fp8",
     "Nvfp4Error", "lib", "library_path",
     "nvfp4_linear_plan", "nvfp4_linear_workspace_bytes", "nvfp4_linear_variant",
     "nvfp4_linear_split_k", "nvfp4_linear_launches_per_run", "nvfp4_linear_run",
@@ -47,6 +48,7 @@ NVFP4_VARIANT_ROW = 4
 NVFP4_PLAN_PDL = 0x10000
 NVFP4_PLAN_EPI_SWIGLU = 0x100
 NVFP4_PLAN_EPI_ARGMAX = 0x200
+NVFP4_PLAN_WEIGHT_FP8 = 0x1000
 NVFP4_PLAN_TEST_STALL = 0x40000000
 NVFP4_STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -66,6 +68,7 @@ EXPORTS = {
     "nvfp4_linear_destroy": (None, [_P]),
     "nvfp4_pack_check": (_c.c_int, [_P, _P, _P, _c.c_int, _c.c_int, _P, _P, _P]),
     "nvfp4_quantize": (_c.c_int, [_P, _c.c_int, _c.c_int, _P, _P, _P, _P, _P]),
+    "nvfp4_quantize_fp8": (_c.c_int, [_P, _c.c_int, _c.c_int, _P, _P, _P, _P]),
     "nvfp4_status_string": (_c.c_char_p, [_c.c_int]),
 }
 
@@ -193,6 +196,13 @@ def nvfp4_quantize(w, N: int, K: int, w_packed, w_scales, w_global, d_bad=None, 
     s = lib().nvfp4_quantize(_ptr(w), N, K, _ptr(w_packed), _ptr(w_scales), _ptr(w_global),
                              _ptr(d_bad), _stream(stream))
     return _check(s, "nvfp4_quantize") if check else s
+
+
+def nvfp4_quantize_fp8(w, N: int, K: int, codes, row_scales, d_bad=None, stream=None,
+                       check: bool = True) -> int:
+    s = lib().nvfp4_quantize_fp8(_ptr(w), N, K, _ptr(codes), _ptr(row_scales), _ptr(d_bad),
+                                 _stream(stream))
+    return _check(s, "nvfp4_quantize_fp8") if check else s
 
 
 def nvfp4_status_string(s: int) -> str:

@@ -32,6 +32,7 @@ struct nvfp4_plan_s {
   unsigned flags;
   int variant;
   int epi;        // fused epilogue: 0 none, 1 SwiGLU, 2 argmax (MMA variant only)
+  int fmt;        // weight format: 0 NVFP4, 1 FP8 (ROW variant only)
   int split_k;
   int num_sms;
   size_t ws_bytes;
@@ -99,7 +100,7 @@ bool lookup_maps(nvfp4_plan_s* p, const void* wp, const void* ws, CUtensorMap* m
   MapEntry& e = p->maps[p->map_next];
   bool ok;
   if (p->variant == int(NVFP4_VARIANT_ROW)) {
-    ok = nvfp4::encode_row_maps(p->N, p->K, p->row.ipu, static_cast<const uint8_t*>(wp),
+    ok = nvfp4::encode_row_maps(p->N, p->K, p->row.ipu, p->row.fmt, static_cast<const uint8_t*>(wp),
                                 static_cast<const uint8_t*>(ws), &e.mw, &e.ms);
   } else {
     const int box_rows = p->variant == int(NVFP4_VARIANT_MMA) ? nvfp4::kMmaTileRows : 128;
@@ -150,6 +151,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   else if (epi_flag == NVFP4_PLAN_EPI_ARGMAX) epi = 2;
   else if (epi_flag != 0u) return NVFP4_ERR_INVALID_ARG;
   if (epi == 1 && N % 2 != 0) return NVFP4_ERR_INVALID_ARG;
+  const int fmt = (flags & NVFP4_PLAN_WEIGHT_FP8) ? 1 : 0;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (device < 0 || device >= ndev) return NVFP4_ERR_INVALID_ARG;
@@ -165,10 +167,11 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   nvfp4_plan_s& p = *h;
   p.M = M; p.N = N; p.K = K; p.device = device; p.flags = flags; p.num_sms = sms;
   p.epi = epi;
+  p.fmt = fmt;
   p.split_k = 1;
   p.ws_bytes = 0;
   unsigned forced = flags & NVFP4_PLAN_VARIANT_MASK;
-  p.variant = forced ? int(forced) : auto_variant(M, N, K);
+  p.variant = forced ? int(forced) : (fmt == 1 ? int(NVFP4_VARIANT_ROW) : auto_variant(M, N, K));
   if (K == 0 || N == 0) {
     // nothing to contract: run() writes zeros (K == 0) or returns (N == 0)
     if (p.variant == int(NVFP4_VARIANT_GEMV) && M > 4) p.variant = int(NVFP4_VARIANT_TC);
@@ -176,6 +179,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   auto configure = [&]() -> nvfp4_status {
     nvfp4_status st = NVFP4_OK;
     if (p.epi != 0 && p.variant != int(NVFP4_VARIANT_MMA)) return NVFP4_ERR_UNSUPPORTED;
+    if (p.fmt != 0 && (p.variant != int(NVFP4_VARIANT_ROW) || p.epi != 0)) return NVFP4_ERR_UNSUPPORTED;
     switch (p.variant) {
       case NVFP4_VARIANT_GEMV: {
         if (M > 4 || size_t(M) * size_t(K) * 4 > 200 * 1024) { st = NVFP4_ERR_UNSUPPORTED; break; }
@@ -196,7 +200,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
       }
       case NVFP4_VARIANT_ROW: {
         if (K == 0 || N == 0) break;
-        p.row.M = M; p.row.N = N; p.row.K = K;
+        p.row.M = M; p.row.N = N; p.row.K = K; p.row.fmt = p.fmt;
         cudaError_t e = nvfp4::row_configure(p.row, sms);
         if (e == cudaSuccess && !nvfp4::tensor_maps_supported()) e = cudaErrorNotSupported;
         if (e == cudaErrorInvalidConfiguration || e == cudaErrorNotSupported) st = NVFP4_ERR_UNSUPPORTED;
@@ -221,14 +225,15 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
     return st;
   };
   nvfp4_status st = configure();
-  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.variant == int(NVFP4_VARIANT_ROW)) {
+  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.fmt == 0 && p.variant == int(NVFP4_VARIANT_ROW)) {
     // the row variant cannot take this shape (X too large to stay resident)
     p.variant = int(NVFP4_VARIANT_MMA);
     p.split_k = 1;
     p.ws_bytes = 0;
     st = configure();
   }
-  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.epi == 0 && p.variant != int(NVFP4_VARIANT_TC)) {
+  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.epi == 0 && p.fmt == 0 &&
+      p.variant != int(NVFP4_VARIANT_TC)) {
     // the automatic choice cannot take this shape: the tcgen05 pipeline can
     p.variant = int(NVFP4_VARIANT_TC);
     p.split_k = 1;
@@ -312,7 +317,8 @@ nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
         if (!lookup_maps(plan, w_packed, w_scales, &mw, &ms)) return NVFP4_ERR_CUDA;
         const bool stall = (plan->flags & NVFP4_PLAN_TEST_STALL) != 0;
         const bool pdl = (plan->flags & NVFP4_PLAN_PDL) != 0;
-        e = nvfp4::launch_row(plan->row, &mw, &ms, w_global, xb, yb, workspace,
+        e = nvfp4::launch_row(plan->row, &mw, &ms, reinterpret_cast<const float*>(w_scales), w_global, xb,
+                              yb, workspace,
                               stall ? kStallTimeoutCycles : kTimeoutCycles, stall, pdl, st);
         break;
       }
@@ -384,6 +390,23 @@ nvfp4_status nvfp4_quantize(const float* w, int N, int K, uint8_t* w_packed, uin
     return NVFP4_ERR_CUDA;
   cudaError_t e = nvfp4::launch_quantize(w, N, K, w_packed, w_scales, w_global, d_bad, sms,
                                          static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status nvfp4_quantize_fp8(const float* w, int N, int K, uint8_t* codes, float* row_scales,
+                                unsigned* d_bad, void* stream) {
+  if (N < 0 || K < 0 || K % 16 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (N > 0 && !row_scales) return NVFP4_ERR_INVALID_ARG;
+  const int64_t n = int64_t(N) * K;
+  if (n > 0 && (!w || !codes)) return NVFP4_ERR_INVALID_ARG;
+  if ((d_bad && !aligned(d_bad, 4)) || (N > 0 && !aligned(row_scales, 16))) return NVFP4_ERR_MISALIGNED;
+  if (n > 0 && (!aligned(w, 16) || !aligned(codes, 16))) return NVFP4_ERR_MISALIGNED;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return NVFP4_ERR_CUDA;
+  cudaError_t e = nvfp4::launch_quantize_fp8(w, N, K, codes, row_scales, d_bad, sms,
+                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 

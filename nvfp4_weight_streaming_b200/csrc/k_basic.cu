@@ -182,6 +182,63 @@ __global__ void k_zero_bf16(uint16_t* y, int64_t count) {
   for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < count; i += stride) y[i] = 0;
 }
 
+// ---------------------------------------------------------------------------
+// FP8 weight tier quantiser: one warp per row. s_n = amax|W[n]| / 448 and
+// code = E4M3_RNE_satfinite(w / s_n), each one fp32 operation; a row with
+// s_n = 0 gets zero codes. Four elements per lane and step (K % 16 == 0).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3x2_from_f32(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__global__ void __launch_bounds__(256)
+k_quantize_fp8_rows(const float* __restrict__ w, int64_t N, int64_t K, uint8_t* __restrict__ codes,
+                    float* __restrict__ row_scales, unsigned* __restrict__ bad) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = int64_t(gridDim.x) * (blockDim.x >> 5);
+  unsigned local_bad = 0;
+  for (int64_t n = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); n < N; n += nw) {
+    const float4* row = reinterpret_cast<const float4*>(w + n * K);
+    float amax = 0.0f;
+    for (int64_t c = lane; c < K / 4; c += 32) {
+      const float4 v = row[c];
+      const float a[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (!isfinite(a[i])) ++local_bad;
+        amax = fmaxf(amax, fabsf(a[i]));
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    const float sn = amax / 448.0f;
+    if (lane == 0) row_scales[n] = sn;
+    uint32_t* out = reinterpret_cast<uint32_t*>(codes + n * K);
+    for (int64_t c = lane; c < K / 4; c += 32) {
+      uint32_t q = 0u;
+      if (sn > 0.0f) {
+        const float4 v = row[c];
+        q = e4m3x2_from_f32(v.x / sn, v.y / sn) | (e4m3x2_from_f32(v.z / sn, v.w / sn) << 16);
+      }
+      out[c] = q;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) local_bad += __shfl_xor_sync(0xffffffffu, local_bad, off);
+  if (lane == 0 && local_bad && bad) atomicAdd(bad, local_bad);
+}
+
+cudaError_t launch_quantize_fp8(const float* w, int64_t N, int64_t K, uint8_t* codes, float* row_scales,
+                                unsigned* bad, int num_sms, cudaStream_t st) {
+  if (N <= 0) return cudaSuccess;
+  const int64_t want = (N + 7) / 8;                       // 8 rows (warps) per block
+  const int grid = int(want < int64_t(num_sms) * 16 ? want : int64_t(num_sms) * 16);
+  k_quantize_fp8_rows<<<grid, 256, 0, st>>>(w, N, K, codes, row_scales, bad);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_zero_bf16(uint16_t* y, int64_t count, cudaStream_t st) {
   if (count <= 0) return cudaSuccess;
   int64_t want = (count + 255) / 256;

@@ -69,11 +69,15 @@ constexpr int ROWS = 16;                         // weight rows per unit
 constexpr int ITEM_K = 512;                      // K elements per item
 constexpr int BOX_W = ROWS * 128;                // codes of 16 rows x 256 elements
 constexpr int BOX_S = ROWS * 16;                 // scales of 16 rows x 256 elements
-constexpr int ITEM_W = 2 * BOX_W;                // 4096 code bytes per item
-constexpr int ITEM_S = 2 * BOX_S;                // 512 scale bytes per item
 constexpr int XPIECE = ITEM_K * 2;               // f16 bytes of one stream per item
 constexpr int XPAD = 64;                         // stream pitch: items * XPIECE + XPAD
-constexpr int IPU_CAP = 10;                      // items per unit at most
+constexpr int IPU_CAP = 10;                      // items per unit at most (NVFP4)
+constexpr int IPU_CAP_FP8 = 5;                   // items per unit at most (FP8: 8 KB per item)
+// Weight formats: NVFP4 (E2M1 codes, E4M3 scale per 16 elements) and the
+// FP8 comparison tier (E4M3 codes [N][K], one fp32 scale per row).
+constexpr int FMT_NVFP4 = 0, FMT_FP8 = 1;
+__host__ __device__ constexpr int item_w_bytes(int fmt) { return fmt == FMT_FP8 ? ROWS * ITEM_K : 2 * ROWS * 128; }
+__host__ __device__ constexpr int item_s_bytes(int fmt) { return fmt == FMT_FP8 ? 0 : 2 * ROWS * 16; }
 constexpr int NST_MAX = 8;                       // ring slots (one unit each)
 constexpr int NST_MIN = 2;
 constexpr int MAX_M = 2;
@@ -92,6 +96,7 @@ struct Params {
   int M, N, K;
   int units16, KS, units, IT, ipu, nst, xstride, sp_row;
   const float* gs;
+  const float* row_scale;     // FP8: per-row scale [N]
   const uint16_t* x;
   uint16_t* y;
   uint32_t* status;
@@ -158,6 +163,7 @@ __device__ __forceinline__ uint32_t xpiece_off(int k) {
 // writes its rows of Y, or, for a K-split unit, its partial and -- if it is
 // the last slice of its row group to finish -- the row group's sum over
 // slices in slice order.
+template <int FMT>
 __device__ __forceinline__ void finish_unit(const Params& p, const float* sPu, int u, int nit, int S,
                                             float fh0, float fh1, float gs, int lane) {
   const int rg = u / p.KS, sl = u - rg * p.KS;
@@ -176,8 +182,11 @@ __device__ __forceinline__ void finish_unit(const Params& p, const float* sPu, i
     v = (vh + vl * (1.0f / 536870912.0f)) * (m == 0 ? fh0 : fh1);
   }
   const int n = rg * ROWS + r;
+  // the output scale: the global scale, times the row's scale for FP8
+  float os = gs;
+  if (FMT == FMT_FP8 && mine && n < p.N) os *= __ldg(p.row_scale + n);
   if (p.KS == 1) {
-    if (mine && n < p.N) p.y[size_t(m) * p.N + n] = float_to_bf16_bits(gs * v);
+    if (mine && n < p.N) p.y[size_t(m) * p.N + n] = float_to_bf16_bits(os * v);
     return;
   }
   float* gp = p.gpart + (size_t(rg) * p.KS) * p.M * ROWS;
@@ -192,14 +201,15 @@ __device__ __forceinline__ void finish_unit(const Params& p, const float* sPu, i
   if (mine) {
     float sum = 0.0f;
     for (int s2 = 0; s2 < p.KS; ++s2) sum += __ldcg(gp + size_t(s2) * p.M * ROWS + m * ROWS + r);
-    if (n < p.N) p.y[size_t(m) * p.N + n] = float_to_bf16_bits(gs * sum);
+    if (n < p.N) p.y[size_t(m) * p.N + n] = float_to_bf16_bits(os * sum);
   }
   if (lane == 0) p.gcnt[rg] = 0u;
 }
 
-// Consumer warp's walk over its items. NT token tiles (2 streams each) per
-// A fragment: S <= 2 streams -> 1, S <= 4 -> 2.
-template <int NT>
+// Consumer warp's walk over its items. NVFP4: NT token tiles (2 streams
+// each) per A fragment, S <= 2 streams -> 1, S <= 4 -> 2. FP8: one tile
+// whose column g is stream g (NT = 1).
+template <int NT, int FMT>
 __device__ __forceinline__ void consume(const Params& p, const uint8_t* sW, const uint8_t* sS,
                                         const uint8_t* sX, float* sP, const int4* meta,
                                         uint32_t* cnt, uint32_t b_full, uint32_t b_empty,
@@ -227,10 +237,53 @@ __device__ __forceinline__ void consume(const Params& p, const uint8_t* sW, cons
       float acc[NT][4];
 #pragma unroll
       for (int tau = 0; tau < NT; ++tau) acc[tau][0] = acc[tau][1] = acc[tau][2] = acc[tau][3] = 0.0f;
-      if (it < p.IT) {                                  // past K: zeros, nothing to add
+      if (FMT == FMT_FP8 && it < p.IT) {
+        // Lane quad t holds elements 16t .. 16t + 15 of each 64-element step:
+        // k slots 2t, 2t+1 <- 4i, 4i+1 and 2t+8, 2t+9 <- 4i+2, 4i+3 of them in
+        // MMA i. Column g of B is stream g; every lane supplies the x of its
+        // quad's elements. The row scale is applied when the unit is done.
+        const uint8_t* ubase = sW + size_t(slot) * ipu * item_w_bytes(FMT);
+        const bool xo = g < S;
+        const uint8_t* xbase = sX + g * p.xstride + it * XPIECE;
+        float da[4] = {0.0f, 0.0f, 0.0f, 0.0f}, db[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          // 128-byte piece 4 s_item + q/2 of the unit; 16 bytes 4 (q & 1) + t of each row
+          const uint8_t* cb = ubase + (4 * s_item + (q >> 1)) * BOX_W;
+          const int sub = 4 * (q & 1) + t;
+          const uint4 w0 = *reinterpret_cast<const uint4*>(cb + g * 128 + ((sub ^ g) << 4));
+          const uint4 w1 = *reinterpret_cast<const uint4*>(cb + (g + 8) * 128 + ((sub ^ g) << 4));
+          const uint32_t r0[4] = {w0.x, w0.y, w0.z, w0.w}, r1[4] = {w1.x, w1.y, w1.z, w1.w};
+          uint32_t h0[8], h1[8];                        // f16x2 of elements (2j, 2j+1)
+#pragma unroll
+          for (int wd = 0; wd < 4; ++wd) {
+            h0[2 * wd] = e4m3x2_to_f16x2(r0[wd]);
+            h0[2 * wd + 1] = e4m3x2_to_f16x2(r0[wd] >> 16);
+            h1[2 * wd] = e4m3x2_to_f16x2(r1[wd]);
+            h1[2 * wd + 1] = e4m3x2_to_f16x2(r1[wd] >> 16);
+          }
+          // x of block 4q + t of the item (16 elements), in the prepared layout
+          const int b = 4 * q + t;
+          uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
+          if (xo) {
+            x0 = *reinterpret_cast<const uint4*>(xbase + (((b & 7) * 2) * 4 + (b >> 3)) * 16);
+            x1 = *reinterpret_cast<const uint4*>(xbase + (((b & 7) * 2 + 1) * 4 + (b >> 3)) * 16);
+          }
+          const uint32_t xr[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (q & 1) mma16816(db, h0[2 * i], h1[2 * i], h0[2 * i + 1], h1[2 * i + 1], xr[2 * i], xr[2 * i + 1]);
+            else mma16816(da, h0[2 * i], h1[2 * i], h0[2 * i + 1], h1[2 * i + 1], xr[2 * i], xr[2 * i + 1]);
+          }
+        }
+        // columns 2t, 2t+1 (streams) of rows g and g + 8
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[0][e] = da[e] + db[e];
+      }
+      if (FMT == FMT_NVFP4 && it < p.IT) {              // past K: zeros, nothing to add
         const int chunk = 2 * s_item + (t >> 1);        // 256-element piece holding blocks 8t..8t+7
-        const uint8_t* box = sW + size_t(slot) * ipu * ITEM_W + chunk * BOX_W;
-        const uint8_t* srow = sS + size_t(slot) * ipu * ITEM_S + chunk * BOX_S + g * 16 + 8 * (t & 1);
+        const uint8_t* box = sW + size_t(slot) * ipu * item_w_bytes(FMT) + chunk * BOX_W;
+        const uint8_t* srow = sS + size_t(slot) * ipu * item_s_bytes(FMT) + chunk * BOX_S + g * 16 + 8 * (t & 1);
         const uint2 sc0 = *reinterpret_cast<const uint2*>(srow);              // row g, blocks 8t..8t+7
         const uint2 sc1 = *reinterpret_cast<const uint2*>(srow + 8 * 16);     // row g + 8
         const uint8_t* xb[NT];
@@ -296,7 +349,7 @@ __device__ __forceinline__ void consume(const Params& p, const uint8_t* sW, cons
             acc[tau][e] += __shfl_xor_sync(0xffffffffu, acc[tau][e], 2);
           }
       }
-      if (t == 0) {
+      if (FMT == FMT_NVFP4 && t == 0) {
         float* e0 = sPu + (size_t(s_item) * ROWS + g) * p.sp_row;
         float* e1 = e0 + 8 * p.sp_row;
 #pragma unroll
@@ -310,6 +363,18 @@ __device__ __forceinline__ void consume(const Params& p, const uint8_t* sW, cons
             }
           }
       }
+      if (FMT == FMT_FP8) {
+        float* e0 = sPu + (size_t(s_item) * ROWS + g) * p.sp_row;
+        float* e1 = e0 + 8 * p.sp_row;
+#pragma unroll
+        for (int sg = 0; sg < 2; ++sg) {
+          const int st = 2 * t + sg;
+          if (st < S) {
+            e0[st] = acc[0][sg];
+            e1[st] = acc[0][2 + sg];
+          }
+        }
+      }
       __syncwarp();
       uint32_t last = 0;
       if (lane == 0) {
@@ -322,7 +387,7 @@ __device__ __forceinline__ void consume(const Params& p, const uint8_t* sW, cons
         // after this warp, like every other, has arrived on its empty barrier)
         __threadfence_block();
         const int nit = min(ipu, p.IT - (u % p.KS) * ipu);
-        finish_unit(p, sPu, u, nit, S, fh0, fh1, gs, lane);
+        finish_unit<FMT>(p, sPu, u, nit, S, fh0, fh1, gs, lane);
         __syncwarp();
         if (lane == 0) cnt[slot] = 0u;
       }
@@ -387,14 +452,15 @@ __device__ __forceinline__ void stage_x(const Params& p, uint8_t* sX, int* emax,
   named_bar(BAR_CONSUMERS, NCT);
 }
 
+template <int FMT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_row(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int nst = p.nst, ipu = p.ipu;
   uint8_t* sW = smem;                                      // nst units of codes (1024-aligned)
-  uint8_t* sS = sW + size_t(nst) * ipu * ITEM_W;           // nst units of scales
-  uint8_t* sX = sS + size_t(nst) * ipu * ITEM_S;           // 2M streams x xstride
+  uint8_t* sS = sW + size_t(nst) * ipu * item_w_bytes(FMT);  // nst units of scales (NVFP4)
+  uint8_t* sX = sS + size_t(nst) * ipu * item_s_bytes(FMT);   // 2M streams x xstride
   float* sP = reinterpret_cast<float*>(sX + size_t(2 * p.M) * p.xstride);
   uint8_t* misc = reinterpret_cast<uint8_t*>(sP) + size_t(nst) * ipu * ROWS * p.sp_row * 4;
   int4* meta = reinterpret_cast<int4*>(misc + MISC_META);
@@ -426,7 +492,7 @@ k_row(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     // -------------------------------------------------------------- producer
     if (lane == 0 && !p.stall) {
       const uint64_t pol = l2_evict_first_policy();
-      const uint32_t unit_bytes = uint32_t(ipu) * (ITEM_W + ITEM_S);
+      const uint32_t unit_bytes = uint32_t(ipu) * (item_w_bytes(FMT) + item_s_bytes(FMT));
       // the first nst units fill the ring without the counter, which belongs
       // to the previous grid until it has completed
       const int nstatic = nst;
@@ -452,10 +518,12 @@ k_row(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
         meta[slot] = make_int4(u, 0, 0, 0);
         mbar_expect_tx(b_full + 8 * slot, unit_bytes);
         // (x, y, z) = (byte in the 128-byte / 16-byte piece, row, piece along K)
-        tma_load_3d_hint(smem_u32(sW + size_t(slot) * ipu * ITEM_W), &tm_w, 0, rg * ROWS, sl * 2 * ipu,
-                         b_full + 8 * slot, pol);
-        tma_load_3d_hint(smem_u32(sS + size_t(slot) * ipu * ITEM_S), &tm_s, 0, rg * ROWS, sl * 2 * ipu,
-                         b_full + 8 * slot, pol);
+        constexpr int PIECES = item_w_bytes(FMT) / BOX_W;   // 128-byte pieces of codes per item row
+        tma_load_3d_hint(smem_u32(sW + size_t(slot) * ipu * item_w_bytes(FMT)), &tm_w, 0, rg * ROWS,
+                         sl * PIECES * ipu, b_full + 8 * slot, pol);
+        if (FMT == FMT_NVFP4)
+          tma_load_3d_hint(smem_u32(sS + size_t(slot) * ipu * item_s_bytes(FMT)), &tm_s, 0, rg * ROWS,
+                           sl * 2 * ipu, b_full + 8 * slot, pol);
         ++j;
       }
       // end marker: every consumer warp passes every unit, so one suffices
@@ -487,10 +555,10 @@ k_row(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     const int S = (*lo_flag ? 2 : 1) * p.M;
     {
       const int cw = warp - 1;
-      if (S <= 2)
-        consume<1>(p, sW, sS, sX, sP, meta, cnt, b_full, b_empty, abort_flag, S, fh0, fh1, gs, cw, lane);
+      if (FMT == FMT_FP8 || S <= 2)
+        consume<1, FMT>(p, sW, sS, sX, sP, meta, cnt, b_full, b_empty, abort_flag, S, fh0, fh1, gs, cw, lane);
       else
-        consume<2>(p, sW, sS, sX, sP, meta, cnt, b_full, b_empty, abort_flag, S, fh0, fh1, gs, cw, lane);
+        consume<2, FMT>(p, sW, sS, sX, sP, meta, cnt, b_full, b_empty, abort_flag, S, fh0, fh1, gs, cw, lane);
     }
   }
   __syncthreads();
@@ -510,6 +578,7 @@ k_row(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
 cudaError_t row_configure(RowConfig& c, int num_sms) {
   using namespace rw;
   if (c.M < 1 || c.M > MAX_M || c.K <= 0 || c.K % 256 != 0 || c.N <= 0) return cudaErrorInvalidConfiguration;
+  if (c.fmt != FMT_NVFP4 && c.fmt != FMT_FP8) return cudaErrorInvalidConfiguration;
   int dev = 0, optin = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -518,7 +587,8 @@ cudaError_t row_configure(RowConfig& c, int num_sms) {
   c.IT = (c.K + ITEM_K - 1) / ITEM_K;
   // K-slices of at most IPU_CAP items, split further while whole-slice units
   // would leave the SMs fewer than eight units each (keeping two items per slice)
-  int KS = (c.IT + IPU_CAP - 1) / IPU_CAP;
+  const int cap = c.fmt == FMT_FP8 ? IPU_CAP_FP8 : IPU_CAP;
+  int KS = (c.IT + cap - 1) / cap;
   while ((long long)c.units16 * KS < 8LL * num_sms && (c.IT + 2 * KS - 1) / (2 * KS) >= 2) KS *= 2;
   c.ipu = (c.IT + KS - 1) / KS;
   c.KS = (c.IT + c.ipu - 1) / c.ipu;               // every slice holds at least one item
@@ -526,7 +596,8 @@ cudaError_t row_configure(RowConfig& c, int num_sms) {
   c.xstride = c.IT * XPIECE + XPAD;
   c.sp_row = 2 * c.M;
   const long long x_bytes = 2LL * c.M * c.xstride;
-  const long long per_slot = (long long)c.ipu * (ITEM_W + ITEM_S) + (long long)c.ipu * ROWS * c.sp_row * 4;
+  const long long per_slot = (long long)c.ipu * (item_w_bytes(c.fmt) + item_s_bytes(c.fmt)) +
+                             (long long)c.ipu * ROWS * c.sp_row * 4;
   const long long left = (long long)optin - 1024 - x_bytes - MISC_BYTES;
   long long nst = left / per_slot;
   if (nst > NST_MAX) nst = NST_MAX;
@@ -542,14 +613,29 @@ cudaError_t row_configure(RowConfig& c, int num_sms) {
   c.ws_gcnt_off = 512;
   c.ws_partials_off = c.ws_gcnt_off + (c.KS > 1 ? ((size_t(c.units16) * 4 + 255) / 256) * 256 : 0);
   c.ws_bytes = c.ws_partials_off + (c.KS > 1 ? ((size_t(c.units16) * c.KS * c.M * ROWS * 4 + 255) / 256) * 256 : 0);
-  return cudaFuncSetAttribute(k_row, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  e = cudaFuncSetAttribute(k_row<FMT_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_row<FMT_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  return e;
 }
 
-bool encode_row_maps(int N, int K, int ipu, const uint8_t* wp, const uint8_t* ws, void* map_w,
+bool encode_row_maps(int N, int K, int ipu, int fmt, const uint8_t* wp, const uint8_t* ws, void* map_w,
                      void* map_s) {
   auto fn = tensor_map_encoder();
   if (!fn) return false;
   const cuuint32_t one[3] = {1, 1, 1};
+  if (fmt == rw::FMT_FP8) {
+    // E4M3 codes [N][K] bytes as (128-byte piece, row, piece along K): boxes
+    // of 128 bytes x 16 rows x 4 ipu pieces, 128-byte swizzle; no scale map
+    const cuuint64_t dim8[3] = {128, cuuint64_t(N), cuuint64_t(K / 128)};
+    const cuuint64_t str8[2] = {cuuint64_t(K), 128};
+    const cuuint32_t box8[3] = {128, uint32_t(rw::ROWS), uint32_t(4 * ipu)};
+    const CUresult r8 = fn(static_cast<CUtensorMap*>(map_w), CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                           const_cast<uint8_t*>(wp), dim8, str8, box8, one, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    *static_cast<CUtensorMap*>(map_s) = *static_cast<CUtensorMap*>(map_w);
+    return r8 == CUDA_SUCCESS;
+  }
   // codes [N][K/2] bytes as (128-byte piece, row, piece along K): boxes of
   // 128 bytes x 16 rows x 2 ipu pieces, 128-byte swizzle
   const cuuint64_t dim_w[3] = {128, cuuint64_t(N), cuuint64_t(K / 256)};
@@ -570,9 +656,9 @@ bool encode_row_maps(int N, int K, int ipu, const uint8_t* wp, const uint8_t* ws
   return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_row(const RowConfig& c, const void* map_w, const void* map_s, const float* gs,
-                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
-                       bool stall, bool pdl, cudaStream_t st) {
+cudaError_t launch_row(const RowConfig& c, const void* map_w, const void* map_s, const float* row_scale,
+                       const float* gs, const uint16_t* x, uint16_t* y, void* workspace,
+                       long long timeout_cycles, bool stall, bool pdl, cudaStream_t st) {
   using namespace rw;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   Params p;
@@ -580,6 +666,7 @@ cudaError_t launch_row(const RowConfig& c, const void* map_w, const void* map_s,
   p.units16 = c.units16; p.KS = c.KS; p.units = c.units; p.IT = c.IT; p.ipu = c.ipu;
   p.nst = c.nst; p.xstride = c.xstride; p.sp_row = c.sp_row;
   p.gs = gs; p.x = x; p.y = y;
+  p.row_scale = row_scale;
   p.status = reinterpret_cast<uint32_t*>(wsb);
   p.claim = reinterpret_cast<uint32_t*>(wsb + c.ws_counters_off);
   p.gcnt = reinterpret_cast<uint32_t*>(wsb + c.ws_gcnt_off);
@@ -596,7 +683,10 @@ cudaError_t launch_row(const RowConfig& c, const void* map_w, const void* map_s,
   cfg.stream = st;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_row, *static_cast<const CUtensorMap*>(map_w),
+  if (c.fmt == FMT_FP8)
+    return cudaLaunchKernelEx(&cfg, k_row<FMT_FP8>, *static_cast<const CUtensorMap*>(map_w),
+                              *static_cast<const CUtensorMap*>(map_s), p);
+  return cudaLaunchKernelEx(&cfg, k_row<FMT_NVFP4>, *static_cast<const CUtensorMap*>(map_w),
                             *static_cast<const CUtensorMap*>(map_s), p);
 }
 

@@ -19,6 +19,10 @@ cudaError_t launch_pack_check(const uint8_t* wp, const uint8_t* ws, const float*
 cudaError_t launch_quantize(const float* w, int64_t N, int64_t K, uint8_t* wp, uint8_t* ws,
                             float* gs, unsigned* bad, int num_sms, cudaStream_t st);
 
+// FP8 tier quantiser: per-row scale amax / 448, E4M3 codes (k_basic.cu).
+cudaError_t launch_quantize_fp8(const float* w, int64_t N, int64_t K, uint8_t* codes, float* row_scales,
+                                unsigned* bad, int num_sms, cudaStream_t st);
+
 // Zero-fill Y (K == 0).
 cudaError_t launch_zero_bf16(uint16_t* y, int64_t count, cudaStream_t st);
 
@@ -79,17 +83,18 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // shared memory by every CTA.
 struct RowConfig {
   int M, N, K;
+  int fmt;   // 0: NVFP4 weights; 1: FP8 weights (E4M3 codes [N][K], fp32 row scales [N])
   int units16, KS, units, IT, ipu, nst, xstride, sp_row, grid;
   size_t smem, ws_counters_off, ws_gcnt_off, ws_partials_off, ws_bytes;
 };
 cudaError_t row_configure(RowConfig& c, int num_sms);
 // TMA descriptors of one weight set for this variant: one box per unit of 16
 // rows x `ipu` 512-element items (codes with the 128-byte swizzle, scales).
-bool encode_row_maps(int N, int K, int ipu, const uint8_t* wp, const uint8_t* ws, void* map_w,
+bool encode_row_maps(int N, int K, int ipu, int fmt, const uint8_t* wp, const uint8_t* ws, void* map_w,
                      void* map_s);
 // One launch.
-cudaError_t launch_row(const RowConfig& c, const void* map_w, const void* map_s, const float* gs,
-                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
-                       bool stall, bool pdl, cudaStream_t st);
+cudaError_t launch_row(const RowConfig& c, const void* map_w, const void* map_s, const float* row_scale,
+                       const float* gs, const uint16_t* x, uint16_t* y, void* workspace,
+                       long long timeout_cycles, bool stall, bool pdl, cudaStream_t st);
 
 }  // namespace nvfp4
