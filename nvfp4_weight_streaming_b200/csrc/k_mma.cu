@@ -135,10 +135,11 @@ __device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned mask, unsign
 
 // Token of accumulator value e of a lane in quad position t, or -1: the
 // columns 2t, 2t+1 of the first token tile (e = 0, 1) and of the second
-// (e = 2, 3; M > 8).
+// (e = 2, 3; M > 8). The block-diagonal class (MC 0) leaves its tokens where
+// class 1 has them.
 template <int MC>
 __device__ __forceinline__ int tok_of(int t, int e) {
-  if (MC == 1) return (t < 2 && e < 2) ? 2 * t + e : -1;
+  if (MC <= 1) return (t < 2 && e < 2) ? 2 * t + e : -1;
   if (e < 2) return 2 * t + e;
   return MC == 3 ? 8 + 2 * t + (e - 2) : -1;
 }
@@ -220,6 +221,16 @@ __device__ __forceinline__ void mma16816(float* c, uint32_t a0, uint32_t a1, uin
       "{%8, %9}, {%0, %1, %2, %3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Same, accumulator starting from zero.
+__device__ __forceinline__ void mma16816_z(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%10, %10, %10, %10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
 // Bounded mbarrier wait. Between checks of the abort flag and the clock the
@@ -443,6 +454,58 @@ __device__ __forceinline__ void compute_step(const uint8_t* sw, const uint8_t* s
   }
 }
 
+// Block-diagonal step (class MC 0: two B streams -- hi and lo plane of one
+// token, or the hi planes of two tokens). The lanes read the same 64
+// elements of rows r and r+8 as in compute_step and MMA i covers the same K
+// slots, but the A fragments are the raw E2M1 values (no scale multiply):
+// B column g is (lane quad g >> 1, stream g & 1) and is nonzero only in that
+// quad's K slots, so after the four MMAs of one scale block per quad (MMA
+// 4j..4j+3 hold elements 16j..16j+15 of lane quad t's 64, i.e. scale block
+// 4t + j of the step), column (t, s) of the product is the exact dot product
+// of one 16-element block of codes with stream s; it is multiplied by that
+// block's E4M3 scale in fp32 and added to the lane's accumulator (set j & 1).
+// bon: this lane supplies B (g >> 1 == t); sxc: its stream's column.
+__device__ __forceinline__ void compute_step_bd(const uint8_t* sw, const uint8_t* ss, int r, float (*acc)[4],
+                                                const uint8_t* sxc, bool bon, uint32_t xg, int t) {
+  const int r1 = r + 8;
+  const uint4 c00 = *reinterpret_cast<const uint4*>(sw + r * 128 + (((2 * t) ^ (r & 7)) << 4));
+  const uint4 c01 = *reinterpret_cast<const uint4*>(sw + r * 128 + (((2 * t + 1) ^ (r & 7)) << 4));
+  const uint4 c10 = *reinterpret_cast<const uint4*>(sw + r1 * 128 + (((2 * t) ^ (r1 & 7)) << 4));
+  const uint4 c11 = *reinterpret_cast<const uint4*>(sw + r1 * 128 + (((2 * t + 1) ^ (r1 & 7)) << 4));
+  const uint32_t s0 = *reinterpret_cast<const uint32_t*>(ss + r * 16 + 4 * t);
+  const uint32_t s1 = *reinterpret_cast<const uint32_t*>(ss + r1 * 16 + 4 * t);
+  const uint32_t w0[8] = {c00.x, c00.y, c00.z, c00.w, c01.x, c01.y, c01.z, c01.w};
+  const uint32_t w1[8] = {c10.x, c10.y, c10.z, c10.w, c11.x, c11.y, c11.z, c11.w};
+  // the four block scales of each row, exactly, in fp32
+  const float2 fa = f16x2_to_float2(e4m3x2_to_f16x2(s0)), fb = f16x2_to_float2(e4m3x2_to_f16x2(s0 >> 16));
+  const float2 fc = f16x2_to_float2(e4m3x2_to_f16x2(s1)), fd = f16x2_to_float2(e4m3x2_to_f16x2(s1 >> 16));
+  const float f0[4] = {fa.x, fa.y, fb.x, fb.y}, f1[4] = {fc.x, fc.y, fd.x, fd.y};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float d[4];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int wd = 2 * j + q;
+      uint32_t h0[4], h1[4];
+      e2m1x8_to_f16x2x4(w0[wd], h0);
+      e2m1x8_to_f16x2x4(w1[wd], h1);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int i = 2 * wd + hh;
+        uint2 bb = make_uint2(0u, 0u);
+        if (bon) bb = *reinterpret_cast<const uint2*>(sxc + xg + 8 * i);
+        if (i % 4 == 0) mma16816_z(d, h0[2 * hh], h1[2 * hh], h0[2 * hh + 1], h1[2 * hh + 1], bb.x, bb.y);
+        else mma16816(d, h0[2 * hh], h1[2 * hh], h0[2 * hh + 1], h1[2 * hh + 1], bb.x, bb.y);
+      }
+    }
+    float* a = acc[j & 1];
+    a[0] = fmaf(f0[j], d[0], a[0]);
+    a[1] = fmaf(f0[j], d[1], a[1]);
+    a[2] = fmaf(f1[j], d[2], a[2]);
+    a[3] = fmaf(f1[j], d[3], a[3]);
+  }
+}
+
 // Consumer warp's walk over the CTA's units. MC = token class (1: M <= 4,
 // 2: M <= 8, 3: M <= 16); NTILE token tiles per A fragment (1: hi and lo in
 // one tile; 2: hi + lo tiles, or two hi tiles; 4: two hi + two lo tiles).
@@ -471,7 +534,8 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
 #pragma unroll
   for (int nt = 0; nt < NTILE; ++nt) {
     int plane, tk;
-    if (MC == 1) { plane = g >> 2; tk = g & 3; }
+    if (MC == 0) { plane = 0; tk = 0; }               // set below
+    else if (MC == 1) { plane = g >> 2; tk = g & 3; }
     else if (MC == 2) { plane = LO ? nt : 0; tk = g; }
     else if (LO) { plane = nt >> 1; tk = 8 * (nt & 1) + g; }
     else { plane = 0; tk = 8 * nt + g; }
@@ -481,6 +545,12 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     const uint32_t cstride = XR ? uint32_t(p.xbox_words * 4) : uint32_t(p.xstride);
     if (LO) xcol[nt] = uint32_t(plane * p.M + (valid ? tk : 0)) * cstride;
     else xcol[nt] = uint32_t(valid ? plane * p.M + tk : p.M) * cstride;
+    if (MC == 0) {
+      // stream g & 1 is column g & 1: hi and lo of token 0 (M = 1) or the hi
+      // planes of tokens 0 and 1 (M = 2, no lo plane)
+      xcol[nt] = uint32_t(g & 1) * cstride;
+      xon[nt] = (g >> 1) == t;
+    }
   }
   float acc[4][4];
 #pragma unroll
@@ -490,7 +560,7 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
   int seg_start = a;
   int nsplit = 0;                                      // split segments handed to the settler
   int tile = a / cnt, j = a - tile * cnt;
-  const int pre_tile = MC == 1 ? prefetch_tile(p, a, b, cnt, L) : -1;
+  const int pre_tile = MC <= 1 ? prefetch_tile(p, a, b, cnt, L) : -1;
   for (int idx = a; idx < b; ++idx) {
     const bool ok = wait_bar(b_full + 8 * st, ph, abort_flag, p, ST_TIMEOUT_CONSUMER);
     if (!__all_sync(0xffffffffu, ok)) break;
@@ -500,9 +570,13 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     constexpr bool EARLY = false;
     // lane t reads 64-element group t of this step (staged X: of the slice)
     const uint32_t xg = uint32_t(XGROUP_BYTES * (XR ? t : 4 * j + t));
-    compute_step<NTILE, EARLY, LO>(sW + st * W_BYTES, sS + st * S_BYTES, r, acc,
-                                   XR ? sX + st * p.xbytes : sX, xcol, xon, xg, t,
-                                   b_empty + 8 * st, lane);
+    if constexpr (MC == 0)
+      compute_step_bd(sW + st * W_BYTES, sS + st * S_BYTES, r, acc, (XR ? sX + st * p.xbytes : sX) + xcol[0],
+                      xon[0], xg, t);
+    else
+      compute_step<NTILE, EARLY, LO>(sW + st * W_BYTES, sS + st * S_BYTES, r, acc,
+                                     XR ? sX + st * p.xbytes : sX, xcol, xon, xg, t,
+                                     b_empty + 8 * st, lane);
     if (!EARLY) {
       __syncwarp();
       if (lane == 0) mbar_arrive(b_empty + 8 * st);
@@ -546,7 +620,27 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     float v[4][2];
 #pragma unroll
     for (int e = 0; e < 4; ++e) v[e][0] = v[e][1] = 0.0f;
-    if (MC == 1) {
+    if (MC == 0) {
+      // block-diagonal: the lanes of a quad hold disjoint blocks of the same
+      // rows; add them (fixed order), then undo the planes' scales
+      float bt[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        bt[e] = at[0][e];
+        bt[e] += __shfl_xor_sync(0xffffffffu, bt[e], 1);
+        bt[e] += __shfl_xor_sync(0xffffffffu, bt[e], 2);
+      }
+      const float h0 = emax[0] == INT_MIN ? 0.0f : ldexpf(1.0f, emax[0] - 14);
+      if (p.M == 1) {
+        const float l0 = h0 * (1.0f / 536870912.0f);          // 2^-LO_SHIFT
+        v[0][0] = bt[0] * h0 + bt[1] * l0;
+        v[0][1] = bt[2] * h0 + bt[3] * l0;
+      } else {
+        const float h1 = emax[1] == INT_MIN ? 0.0f : ldexpf(1.0f, emax[1] - 14);
+        v[0][0] = bt[0] * h0; v[1][0] = bt[1] * h1;
+        v[0][1] = bt[2] * h0; v[1][1] = bt[3] * h1;
+      }
+    } else if (MC == 1) {
       // one tile: columns 0..3 hi tokens 0..3, 4..7 lo tokens 0..3; lo partner lane t^2
       float o[4];
 #pragma unroll
@@ -591,7 +685,7 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     }
     const int ord = bnd_in(tcur * cnt, this_start, L, p.P);
     bool done_here = false;
-    if (MC == 1 && tcur == pre_tile && ord == 0 && idx + 1 == b &&
+    if (MC <= 1 && tcur == pre_tile && ord == 0 && idx + 1 == b &&
         __all_sync(0xffffffffu, *pre_flag != 0u)) {
       // the settler has copied the other piece into shared memory
       __threadfence_block();
@@ -875,7 +969,8 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
       bool need_lo = false;
       for (int m = 0; m < p.M; ++m) need_lo |= p.xlo[m] != 0u;
       if constexpr (MC == 1) {
-        if (need_lo) NVFP4_CONSUME(1, 1, true, true, p.xemax); else NVFP4_CONSUME(1, 1, false, true, p.xemax);
+        if (p.M == 1 || (p.M == 2 && !need_lo)) NVFP4_CONSUME(0, 1, false, true, p.xemax);
+        else if (need_lo) NVFP4_CONSUME(1, 1, true, true, p.xemax); else NVFP4_CONSUME(1, 1, false, true, p.xemax);
       } else if constexpr (MC == 2) {
         if (need_lo) NVFP4_CONSUME(2, 2, true, true, p.xemax); else NVFP4_CONSUME(2, 1, false, true, p.xemax);
       } else if constexpr (MC == 3) {
@@ -940,7 +1035,8 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     const bool need_lo = flags[0] != 0u;
 
     if constexpr (MC == 1) {
-      if (need_lo) NVFP4_CONSUME(1, 1, true, false, emax); else NVFP4_CONSUME(1, 1, false, false, emax);
+      if (p.M == 1 || (p.M == 2 && !need_lo)) NVFP4_CONSUME(0, 1, false, false, emax);
+      else if (need_lo) NVFP4_CONSUME(1, 1, true, false, emax); else NVFP4_CONSUME(1, 1, false, false, emax);
     } else if constexpr (MC == 2) {
       if (need_lo) NVFP4_CONSUME(2, 2, true, false, emax); else NVFP4_CONSUME(2, 1, false, false, emax);
     } else {
