@@ -94,6 +94,7 @@ constexpr uint32_t ST_TIMEOUT_PRODUCER = 1u, ST_TIMEOUT_CONSUMER = 2u, ST_TIMEOU
 
 struct Params {
   int M, N, K, tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, nstage;
+  int tpc;                                   // whole tiles per CTA (no split tiles), 0: stream-K
   int xbytes, xbox_words, xbox_bytes;        // X in the ring: stage area, words per column, box bytes
   const int* xemax;                          // X in the ring: per-token exponent maximum
   const uint32_t* xlo;                       // X in the ring: per-token "lo plane used"
@@ -882,7 +883,9 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
   const int ks0 = s * p.ks_base + min(s, p.ks_rem);
   const int klen = cnt * KS, k0e = ks0 * KS;
   const int L = p.tiles * cnt;
-  const int a = int((long long)c * L / p.P), b = int((long long)(c + 1) * L / p.P);
+  // whole tiles per CTA (tpc > 0), else an even share of the units (stream-K)
+  const int a = p.tpc > 0 ? min(c * p.tpc, p.tiles) * cnt : int((long long)c * L / p.P);
+  const int b = p.tpc > 0 ? min((c + 1) * p.tpc, p.tiles) * cnt : int((long long)(c + 1) * L / p.P);
 
   // Dependent launches (PDL) may start now: they only stream weights until
   // this grid has completed.
@@ -1149,13 +1152,25 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   const int ks_base = ksteps / S, ks_rem = ksteps % S;
   const long long min_units = (long long)c.tiles * ks_base;
   if (P > min_units) P = int(min_units);
+  // One whole tile per CTA when there are at most as many tiles as SMs and
+  // they keep at least 85% of the SMs busy: a split tile costs its pieces a
+  // round trip through the workspace and the CTA holding the last piece a
+  // wait at the end of the call, which measured more than the idle SMs
+  // (decode projection, N = 34816: 136 tiles on 136 SMs, 20 us per call
+  // against 23 with stream-K on 148; M = 16: 29 against 36). With several
+  // tiles per CTA (lm_head) stream-K over all SMs measured faster.
+  c.tpc = 0;
+  if (S == 1 && c.tiles <= num_sms && c.tiles * 100 >= num_sms * 85) {
+    c.tpc = 1;
+    P = c.tiles;
+  }
   c.S = S; c.P = P; c.ks_base = ks_base; c.ks_rem = ks_rem;
   c.grid = S * P;
   c.xk_max = (ks_base + (ks_rem ? 1 : 0)) * KS;
   c.xstride = c.xr ? c.x_box : stride_for(c.xk_max / KS);
   int pmax = 1;
   bool split = S > 1;
-  for (int s = 0; s < S; ++s) {
+  for (int s = 0; s < S && c.tpc == 0; ++s) {
     const int cnt = ks_base + (s < ks_rem ? 1 : 0);
     const long long L = (long long)c.tiles * cnt;
     std::vector<int> pieces(c.tiles, 1);
@@ -1209,7 +1224,7 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
   Params p;
   p.M = c.M; p.N = c.N; p.K = c.K; p.tiles = c.tiles; p.S = c.S; p.P = c.P;
   p.ks_base = c.ks_base; p.ks_rem = c.ks_rem; p.ncols = c.ncols; p.xk_max = c.xk_max;
-  p.xstride = c.xstride; p.pmax = c.pmax; p.nstage = c.nstage;
+  p.xstride = c.xstride; p.pmax = c.pmax; p.nstage = c.nstage; p.tpc = c.tpc;
   p.xbytes = c.xbytes; p.xbox_words = c.x_box / 4; p.xbox_bytes = c.ncols * c.x_box;
   p.gs = gs; p.x = x; p.y = y;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);

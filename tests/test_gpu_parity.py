@@ -178,7 +178,10 @@ def test_linear_tiny_all_variants(M):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 520, 512), (3, 1000, 768), (5, 129, 256), (16, 777, 1280),
-                                   (2, 1, 256), (9, 4097, 512)])
+                                   (2, 1, 256), (9, 4097, 512),
+                                   # 130 and 128 tiles of 256 rows: one whole tile per CTA
+                                   (1, 130 * 256 - 77, 512), (2, 130 * 256 - 77, 512),
+                                   (16, 127 * 256 + 5, 256)])
 def test_linear_ragged_shapes(M, N, K):
     """N not a multiple of any tile; several tiles plus a ragged tail."""
     W = synth.normal_f32(N * K, 0.02, seed=3, stream=7).reshape(N, K)
