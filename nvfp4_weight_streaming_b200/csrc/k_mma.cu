@@ -982,8 +982,20 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     } else {
     const int ctid = threadIdx.x - 32;                    // 0 .. NCW*32-1
     constexpr int NCT = NCW * 32;
-    const int chunks = klen / 8;
-    const int nreal = p.M * chunks;
+    // Only the K-steps of the slice that this CTA's units touch are staged:
+    // nx_steps of them, circularly from step j0x (a range shorter than a
+    // tile's K either lies in one tile or wraps from the end of one tile to
+    // the start of the next). The exponent maximum is taken over them too:
+    // the planes' scales are undone before any sum leaves the CTA.
+    const int nx_steps = min(cnt, b - a), j0x = a % cnt;
+    const int nx = nx_steps * (KS / 8);                  // 16-byte chunks per token
+    auto chunk_of = [&](int rem) {
+      int st = j0x + (rem >> 5);
+      if (st >= cnt) st -= cnt;
+      return st * (KS / 8) + (rem & 31);
+    };
+    static_assert(KS / 8 == 32, "chunk_of: 32 chunks of 8 elements per K-step");
+    const int nreal = p.M * nx;
     // 1. X slice -> shared memory as raw bf16, in the hi plane's places, and
     //    the per-token exponent maximum (lanes holding the same token reduce
     //    in the warp: one shared-memory atomic per token and warp)
@@ -995,8 +1007,8 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
         const int u = base + (ctid & 31) + h * NCT;
         mm[h] = -1;
         if (u < nreal) {
-          mm[h] = u / chunks;
-          kk[h] = u - mm[h] * chunks;
+          mm[h] = u / nx;
+          kk[h] = chunk_of(u - mm[h] * nx);
           xv[h] = *reinterpret_cast<const uint4*>(p.x + size_t(mm[h]) * p.K + k0e + 8 * kk[h]);
         }
       }
@@ -1019,7 +1031,7 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     bool lo_used = false;
 #pragma unroll 1
     for (int u = ctid; u < nreal; u += NCT) {
-      const int m = u / chunks, kc = u - m * chunks;
+      const int m = u / nx, kc = chunk_of(u - m * nx);
       const int sh = (emax[m] == INT_MIN) ? 0 : 14 - emax[m];
       const uint32_t o0 = x_off(8 * kc), o1 = x_off(8 * kc + 4);
       uint8_t* ch = sX + size_t(m) * p.xstride;
