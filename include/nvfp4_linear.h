@@ -154,10 +154,20 @@ size_t nvfp4_linear_workspace_bytes(nvfp4_plan_t plan);
 int nvfp4_linear_variant(nvfp4_plan_t plan);
 int nvfp4_linear_split_k(nvfp4_plan_t plan);
 
+/* The variant an AUTO plan of this shape starts from: the fastest measured
+ * variant of the nearest shape in the library's table of per-variant times
+ * on B200 (nearest: smallest 2 |log2 M - log2 Mt| + |log2 NK - log2 NtKt|,
+ * the first such row on a tie). nvfp4_linear_plan then falls back to the
+ * MMA variant, and from there to TC, if that variant cannot take the shape,
+ * the epilogue or the weight format. -1 for M outside [1,16], negative N/K
+ * or K % 256 != 0. Host-only; touches no device. */
+int nvfp4_auto_variant(int M, int N, int K);
+
 /* Kernels one nvfp4_linear_run (or nvfp4_linear_run_static) of this plan
- * launches: 2 for the mma variant with M >= 5 (X is converted to its two f16
- * planes by a kernel of its own first), 1 otherwise, 0 when N == 0; -1 if the
- * plan is null. Host-only; touches no device. */
+ * launches: 2 for the mma variant when X goes through its ring (M >= 5, or a
+ * K so long that X does not fit next to the ring: X is converted to its two
+ * f16 planes by a kernel of its own first), 1 otherwise, 0 when N == 0; -1
+ * if the plan is null. Host-only; touches no device. */
 int nvfp4_linear_launches_per_run(nvfp4_plan_t plan);
 
 /* Run the linear on `stream` (device pointers, see the layout above):

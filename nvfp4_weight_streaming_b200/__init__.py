@@ -24,7 +24,7 @@ __all__ = [
     "NVFP4_PLAN_PDL", "NVFP4_PLAN_TEST_STALL", "NVFP4_PLAN_EPI_SWIGLU", "NVFP4_PLAN_EPI_ARGMAX",
     "NVFP4_PLAN_WEIGHT_FP8", "nvfp4_quantize_fp8",
     "Nvfp4Error", "lib", "library_path",
-    "nvfp4_linear_plan", "nvfp4_linear_workspace_bytes", "nvfp4_linear_variant",
+    "nvfp4_linear_plan", "nvfp4_auto_variant", "nvfp4_linear_workspace_bytes", "nvfp4_linear_variant",
     "nvfp4_linear_split_k", "nvfp4_linear_launches_per_run", "nvfp4_linear_run",
     "nvfp4_linear_run_static",
     "NVFP4_STATIC_SCRATCH_BYTES", "nvfp4_linear_status", "nvfp4_linear_destroy",
@@ -58,6 +58,7 @@ _P = _c.c_void_p
 EXPORTS = {
     "nvfp4_linear_plan": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_uint,
                                      _c.POINTER(_P)]),
+    "nvfp4_auto_variant": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int]),
     "nvfp4_linear_workspace_bytes": (_c.c_size_t, [_P]),
     "nvfp4_linear_variant": (_c.c_int, [_P]),
     "nvfp4_linear_split_k": (_c.c_int, [_P]),
@@ -146,6 +147,11 @@ def nvfp4_linear_workspace_bytes(plan) -> int:
 
 def nvfp4_linear_variant(plan) -> int:
     return int(lib().nvfp4_linear_variant(plan))
+
+
+def nvfp4_auto_variant(M: int, N: int, K: int) -> int:
+    """Variant an AUTO plan of this shape starts from (host-only query)."""
+    return int(lib().nvfp4_auto_variant(M, N, K))
 
 
 def nvfp4_linear_split_k(plan) -> int:

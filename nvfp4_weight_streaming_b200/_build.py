@@ -30,6 +30,7 @@ def sources():
 def inputs():
     return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh")) +
                               glob.glob(os.path.join(CSRC, "*.h")) +
+                              glob.glob(os.path.join(CSRC, "*.csv")) +
                               glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
@@ -43,6 +44,9 @@ def stale() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not stale():
         return LIB
+    # the AUTO variant table compiled into api.cu
+    from . import gen_variant_table
+    gen_variant_table.generate()
     nvcc = os.environ.get("NVCC", "nvcc")
     tmp = LIB + ".tmp%d" % os.getpid()
     cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]

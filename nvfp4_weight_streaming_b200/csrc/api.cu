@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 #include <cstdlib>
+#include <cmath>
 #include <mutex>
 #include <new>
 
@@ -77,14 +78,28 @@ nvfp4_status static_scratch_address(int device, void** out) {
   return NVFP4_OK;
 }
 
-// Which variant AUTO takes for a shape. Measured on B200 for the 5120 x 34816
-// projection, the TMA + warp-MMA pipeline is fastest for every M in 1..16
-// (M = 1: 24.8 us against 37.7 for the CUDA-core GEMV; M = 16: 36.3 us
-// against 105.9 for tcgen05); plan() falls back to tcgen05 for shapes it
-// cannot take.
+// Which variant AUTO takes for a shape: the fastest measured variant of the
+// nearest shape in the table measured on B200 (variant_table.csv, written
+// by tune_variants.py; variant_table.inc is generated from it at build
+// time). Nearest: the smallest 2 |log2 M - log2 Mt| + |log2 NK - log2 NtKt|,
+// the first such row on a tie. plan() falls back to the MMA pipeline, then
+// to tcgen05, when the chosen variant cannot take the shape.
+struct TableRow { int M, N, K, variant; };
+constexpr TableRow kVariantTable[] = {
+#include "variant_table.inc"
+};
+
 int auto_variant(int M, int N, int K) {
-  (void)M; (void)N; (void)K;
-  return int(NVFP4_VARIANT_MMA);
+  if (M < 1 || N < 1 || K < 1) return int(NVFP4_VARIANT_MMA);
+  const double lm = std::log2(double(M)), lnk = std::log2(double(N)) + std::log2(double(K));
+  double best = 1e300;
+  int v = int(NVFP4_VARIANT_MMA);
+  for (const TableRow& r : kVariantTable) {
+    const double d = 2.0 * std::fabs(lm - std::log2(double(r.M))) +
+                     std::fabs(lnk - std::log2(double(r.N)) - std::log2(double(r.K)));
+    if (d < best) { best = d; v = r.variant; }
+  }
+  return v;
 }
 
 // Copy of the TMA descriptors for (wp, ws), encoding them on first use.
@@ -225,8 +240,9 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
     return st;
   };
   nvfp4_status st = configure();
-  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.fmt == 0 && p.variant == int(NVFP4_VARIANT_ROW)) {
-    // the row variant cannot take this shape (X too large to stay resident)
+  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.fmt == 0 && p.variant != int(NVFP4_VARIANT_MMA) &&
+      p.variant != int(NVFP4_VARIANT_TC)) {
+    // the table's choice (GEMV, row) cannot take this shape or epilogue
     p.variant = int(NVFP4_VARIANT_MMA);
     p.split_k = 1;
     p.ws_bytes = 0;
@@ -244,6 +260,11 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   if (st != NVFP4_OK) { delete h; return st; }
   *out = h;
   return NVFP4_OK;
+}
+
+int nvfp4_auto_variant(int M, int N, int K) {
+  if (M < 1 || M > 16 || N < 0 || K < 0 || K % 256 != 0) return -1;
+  return auto_variant(M, N, K);
 }
 
 size_t nvfp4_linear_workspace_bytes(nvfp4_plan_t plan) { return plan ? plan->ws_bytes : 0; }
