@@ -38,9 +38,10 @@ FALLBACK_HBM_GBS = 6650.0
 
 def bytes_per_call(M: int, N: int, K: int, fmt: str = "nvfp4", epi: str = "none") -> int:
     """Algorithmic bytes of one call: weights (NVFP4 codes and E4M3 scales, or
-    FP8 codes and fp32 row scales), X, and the output (Y; N/2 columns with the
-    SwiGLU epilogue; an int32 index and a float value per token with argmax)."""
-    wbytes = N * K // 2 + N * K // 16 if fmt == "nvfp4" else N * K + 4 * N
+    FP8 codes and fp32 row scales), X (bf16; the W4A4 tier quantises it in the
+    kernel), and the output (Y; N/2 columns with the SwiGLU epilogue; an int32
+    index and a float value per token with argmax)."""
+    wbytes = N * K // 2 + N * K // 16 if fmt in ("nvfp4", "w4a4") else N * K + 4 * N
     out = {"none": 2 * M * N, "swiglu": M * N, "argmax": 8 * M}[epi]
     return wbytes + 2 * M * K + out
 
@@ -178,7 +179,8 @@ def aggregate(world: int, bytes_per_call: float, sec_per_call_this_rank: float):
 
 class Problem:
     """One workload on the device: weight copies, X, Y, plan, workspace.
-    fmt "nvfp4" (the method) or "fp8" (the comparison tier); epi "none",
+    fmt "nvfp4" (the method), "w4a4" (NVFP4 weights, X quantised to NVFP4 in the
+    kernel) or "fp8" (the comparison tier); epi "none",
     "swiglu" or "argmax" (fused epilogues)."""
 
     def __init__(self, name: str, M: int, variant: int, min_footprint: float, flags: int = 0,
@@ -195,7 +197,9 @@ class Problem:
         # weights: generated on the host, quantised on the device by the library
         W = torch.from_numpy(synth.weights_f32(wl)).cuda()
         bad = torch.zeros(1, dtype=torch.int32, device="cuda")
-        if fmt == "nvfp4":
+        if fmt in ("nvfp4", "w4a4"):
+            if fmt == "w4a4":
+                flags |= nv.NVFP4_PLAN_ACT_NVFP4
             packed = torch.empty((self.N, self.K // 2), dtype=torch.uint8, device="cuda")
             scales = torch.empty((self.N, self.K // 16), dtype=torch.uint8, device="cuda")
             gs = torch.empty(1, dtype=torch.float32, device="cuda")
@@ -436,14 +440,18 @@ def run_ours(args):
                  [("verify", m, "nvfp4", "swiglu") for m in (1, 16)] + \
                  [("lm_head", m, "nvfp4", "argmax") for m in (1, 16)] + \
                  [("verify", m, "fp8", "none") for m in (1, 2)] + \
-                 [("down", 1, "fp8", "none"), ("lm_head", 1, "fp8", "none")]
+                 [("down", 1, "fp8", "none"), ("lm_head", 1, "fp8", "none")] + \
+                 [("verify", m, "w4a4", "none") for m in (1, 4)] + [("down", 1, "w4a4", "none")]
         base_us = {}
         for (name, M, fmt, epi) in points:
             v = variant if (fmt == "nvfp4" and epi == "none") else 0
             q = Problem(name, M, v, min_footprint=4.2 * l2, flags=flags, fmt=fmt, epi=epi)
             s2, _, r2 = time_problem(q, max(args.steps, 200), args.warmup, world, repeats=args.repeats)
             g = effective_gbs(q.bytes, s2)
-            pt = {"workload": name, "M": M, "N": q.N, "K": q.K, "weights": fmt, "epilogue": epi,
+            pt = {"workload": name, "M": M, "N": q.N, "K": q.K,
+                  "weights": "nvfp4" if fmt == "w4a4" else fmt,
+                  "activations": "nvfp4 (quantised in the kernel)" if fmt == "w4a4" else "bf16",
+                  "epilogue": epi,
                   "variant": VARIANT_NAMES[q.variant], "split_k": q.split_k,
                   "bytes_per_call": q.bytes, "us_per_call": s2 * 1e6,
                   "us_spread": [min(r2) * 1e6, max(r2) * 1e6], "GBps": g,

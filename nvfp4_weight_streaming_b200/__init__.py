@@ -22,7 +22,7 @@ __all__ = [
     "NVFP4_VARIANT_AUTO", "NVFP4_VARIANT_GEMV", "NVFP4_VARIANT_MMA", "NVFP4_VARIANT_TC",
     "NVFP4_VARIANT_ROW",
     "NVFP4_PLAN_PDL", "NVFP4_PLAN_TEST_STALL", "NVFP4_PLAN_EPI_SWIGLU", "NVFP4_PLAN_EPI_ARGMAX",
-    "NVFP4_PLAN_WEIGHT_FP8", "nvfp4_quantize_fp8",
+    "NVFP4_PLAN_WEIGHT_FP8", "NVFP4_PLAN_ACT_NVFP4", "nvfp4_quantize_fp8",
     "Nvfp4Error", "lib", "library_path",
     "nvfp4_linear_plan", "nvfp4_auto_variant", "nvfp4_linear_workspace_bytes", "nvfp4_linear_variant",
     "nvfp4_linear_split_k", "nvfp4_linear_launches_per_run", "nvfp4_linear_run",
@@ -49,6 +49,7 @@ NVFP4_PLAN_PDL = 0x10000
 NVFP4_PLAN_EPI_SWIGLU = 0x100
 NVFP4_PLAN_EPI_ARGMAX = 0x200
 NVFP4_PLAN_WEIGHT_FP8 = 0x1000
+NVFP4_PLAN_ACT_NVFP4 = 0x2000
 NVFP4_PLAN_TEST_STALL = 0x40000000
 NVFP4_STATIC_SCRATCH_BYTES = 16 << 20
 

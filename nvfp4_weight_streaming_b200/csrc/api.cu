@@ -34,6 +34,7 @@ struct nvfp4_plan_s {
   int variant;
   int epi;        // fused epilogue: 0 none, 1 SwiGLU, 2 argmax (MMA variant only)
   int fmt;        // weight format: 0 NVFP4, 1 FP8 (ROW variant only)
+  int act4;       // W4A4: X quantised to NVFP4 in the kernel (MMA variant, staged X)
   int split_k;
   int num_sms;
   size_t ws_bytes;
@@ -167,6 +168,8 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   else if (epi_flag != 0u) return NVFP4_ERR_INVALID_ARG;
   if (epi == 1 && N % 2 != 0) return NVFP4_ERR_INVALID_ARG;
   const int fmt = (flags & NVFP4_PLAN_WEIGHT_FP8) ? 1 : 0;
+  const int act4 = (flags & NVFP4_PLAN_ACT_NVFP4) ? 1 : 0;
+  if (act4 && fmt) return NVFP4_ERR_UNSUPPORTED;
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess) return NVFP4_ERR_CUDA;
   if (device < 0 || device >= ndev) return NVFP4_ERR_INVALID_ARG;
@@ -183,10 +186,12 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   p.M = M; p.N = N; p.K = K; p.device = device; p.flags = flags; p.num_sms = sms;
   p.epi = epi;
   p.fmt = fmt;
+  p.act4 = act4;
   p.split_k = 1;
   p.ws_bytes = 0;
   unsigned forced = flags & NVFP4_PLAN_VARIANT_MASK;
-  p.variant = forced ? int(forced) : (fmt == 1 ? int(NVFP4_VARIANT_ROW) : auto_variant(M, N, K));
+  p.variant = forced ? int(forced)
+                     : (fmt == 1 ? int(NVFP4_VARIANT_ROW) : act4 ? int(NVFP4_VARIANT_MMA) : auto_variant(M, N, K));
   if (K == 0 || N == 0) {
     // nothing to contract: run() writes zeros (K == 0) or returns (N == 0)
     if (p.variant == int(NVFP4_VARIANT_GEMV) && M > 4) p.variant = int(NVFP4_VARIANT_TC);
@@ -195,6 +200,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
     nvfp4_status st = NVFP4_OK;
     if (p.epi != 0 && p.variant != int(NVFP4_VARIANT_MMA)) return NVFP4_ERR_UNSUPPORTED;
     if (p.fmt != 0 && (p.variant != int(NVFP4_VARIANT_ROW) || p.epi != 0)) return NVFP4_ERR_UNSUPPORTED;
+    if (p.act4 && p.variant != int(NVFP4_VARIANT_MMA)) return NVFP4_ERR_UNSUPPORTED;
     switch (p.variant) {
       case NVFP4_VARIANT_GEMV: {
         if (M > 4 || size_t(M) * size_t(K) * 4 > 200 * 1024) { st = NVFP4_ERR_UNSUPPORTED; break; }
@@ -204,7 +210,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
       }
       case NVFP4_VARIANT_MMA: {
         if (K == 0 || N == 0) break;
-        p.mma.M = M; p.mma.N = N; p.mma.K = K; p.mma.epi = p.epi;
+        p.mma.M = M; p.mma.N = N; p.mma.K = K; p.mma.epi = p.epi; p.mma.act4 = p.act4;
         cudaError_t e = nvfp4::mma_configure(p.mma, sms);
         if (e == cudaSuccess && !nvfp4::tensor_maps_supported()) e = cudaErrorNotSupported;
         if (e == cudaErrorInvalidConfiguration || e == cudaErrorNotSupported) st = NVFP4_ERR_UNSUPPORTED;
@@ -248,7 +254,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
     p.ws_bytes = 0;
     st = configure();
   }
-  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.epi == 0 && p.fmt == 0 &&
+  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.epi == 0 && p.fmt == 0 && p.act4 == 0 &&
       p.variant != int(NVFP4_VARIANT_TC)) {
     // the automatic choice cannot take this shape: the tcgen05 pipeline can
     p.variant = int(NVFP4_VARIANT_TC);

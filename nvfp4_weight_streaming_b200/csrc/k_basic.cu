@@ -97,27 +97,6 @@ k_amax(const float* __restrict__ w, int64_t n, unsigned* __restrict__ amax_bits,
   }
 }
 
-// E4M3 round-to-nearest-even with saturation (hardware conversion); the
-// result's low byte is the code of `u`.
-__device__ __forceinline__ uint32_t e4m3_rne_sat(float u) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(u));
-  return r & 0xFFu;
-}
-
-// Two E2M1 codes (RNE, saturating): `lo` in bits 0..3, `hi` in bits 4..7.
-// A code of magnitude 0 is stored as 0x0 (no negative zero).
-__device__ __forceinline__ uint32_t e2m1x2_rne_sat(float lo, float hi) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 t;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
-      "cvt.u32.u8 %0, t;\n\t}"
-      : "=r"(r) : "f"(hi), "f"(lo));
-  if ((r & 0x07u) == 0) r &= 0xF0u;
-  if ((r & 0x70u) == 0) r &= 0x0Fu;
-  return r;
-}
-
 __global__ void __launch_bounds__(256)
 k_quantize_blocks(const float* __restrict__ w, int64_t nblocks, const unsigned* __restrict__ amax_bits,
                   uint8_t* __restrict__ wp, uint8_t* __restrict__ ws) {
@@ -132,23 +111,8 @@ k_quantize_blocks(const float* __restrict__ w, int64_t nblocks, const unsigned* 
       float4 t = src[i];
       v[4 * i] = t.x; v[4 * i + 1] = t.y; v[4 * i + 2] = t.z; v[4 * i + 3] = t.w;
     }
-    float amax_b = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
-    const float t = __fdiv_rn(amax_b, 6.0f);
-    const float u = (gs > 0.0f) ? __fdiv_rn(t, gs) : 0.0f;
-    const uint32_t s_code = e4m3_rne_sat(u);
-    const float ds = __half2float(__ushort_as_half(
-        static_cast<unsigned short>(e4m3x2_to_f16x2(s_code) & 0xFFFFu)));
-    const float denom = __fmul_rn(ds, gs);
-    uint32_t packed[2] = {0u, 0u};
-    if (denom > 0.0f) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint32_t byte = e2m1x2_rne_sat(__fdiv_rn(v[2 * j], denom), __fdiv_rn(v[2 * j + 1], denom));
-        packed[j / 4] |= byte << (8 * (j % 4));
-      }
-    }
+    uint32_t s_code, packed[2];
+    quantize_block16(v, gs, s_code, packed);
     *reinterpret_cast<uint2*>(wp + 8 * b) = make_uint2(packed[0], packed[1]);
     ws[b] = static_cast<uint8_t>(s_code);
   }

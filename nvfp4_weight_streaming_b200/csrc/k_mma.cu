@@ -82,9 +82,11 @@ constexpr int MISC_BASE = 1024;            // barriers, flags, lists
 inline int misc_bytes(int M) { return MISC_BASE + (M <= 4 ? M * TROWS * 4 : 0); }
 // misc area: barriers [0,256) (full, empty, qfull, qempty: 8 each), emax [256,320),
 // flags [320,336) (need_lo, abort, list count), skip masks [336,368),
-// piece slots [384,640), end-phase list [640,896)
+// prefetch flag [368,372), W4A4 amax and gs_x [372,380), piece slots
+// [384,640), end-phase list [640,896)
 constexpr int MISC_EMAX = 256, MISC_FLAGS = 320, MISC_SKIP = 336, MISC_PREFLAG = 368, MISC_PIECES = 384,
-              MISC_LIST = 640, MISC_PREBUF = 1024;   // prefetched piece: [M <= 4][TROWS] floats
+              MISC_LIST = 640, MISC_PREBUF = 1024,   // prefetched piece: [M <= 4][TROWS] floats
+              MISC_XAMAX = 372, MISC_XGS = 376;      // W4A4: largest |x| (bf16 bits), gs_x
 constexpr int LO_SHIFT = X_LO_SHIFT;
 constexpr int BAR_CONSUMERS = 1;           // named barrier of the consumer warps
 constexpr int XR_MIN_M = 5;                // token counts from which X goes through the ring
@@ -95,6 +97,7 @@ constexpr uint32_t ST_TIMEOUT_PRODUCER = 1u, ST_TIMEOUT_CONSUMER = 2u, ST_TIMEOU
 struct Params {
   int M, N, K, tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, nstage;
   int tpc;                                   // whole tiles per CTA (no split tiles), 0: stream-K
+  int act4;                                  // W4A4: X quantised to NVFP4 in the kernel
   int xbytes, xbox_words, xbox_bytes;        // X in the ring: stage area, words per column, box bytes
   const int* xemax;                          // X in the ring: per-token exponent maximum
   const uint32_t* xlo;                       // X in the ring: per-token "lo plane used"
@@ -669,6 +672,13 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
         v[2 + e][1] = at[1 % NTILE][2 + e] * fh[2 + e] + l3 * fl[2 + e];
       }
     }
+    if (p.act4) {
+      // W4A4: the per-tensor scale of the quantised X (staged X: emax sits in
+      // the CTA's misc area next to it)
+      const float gsx = *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(emax) - MISC_EMAX + MISC_XGS);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) { v[e][0] *= gsx; v[e][1] *= gsx; }
+    }
     const int this_start = seg_start;
     seg_start = idx + 1;
     const bool whole = (p.S == 1) && (this_start == tcur * cnt) && (jcur + 1 == cnt);
@@ -896,6 +906,7 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     for (int m = 0; m < 16; ++m) emax[m] = INT_MIN;
     flags[0] = 0u; flags[1] = 0u; flags[2] = 0u;
     *pre_flag = 0u;
+    *reinterpret_cast<uint32_t*>(misc + MISC_XAMAX) = 0u;
     for (int i = 0; i < QN; ++i) skip[i] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -996,6 +1007,7 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     };
     static_assert(KS / 8 == 32, "chunk_of: 32 chunks of 8 elements per K-step");
     const int nreal = p.M * nx;
+    if (!p.act4) {
     // 1. X slice -> shared memory as raw bf16, in the hi plane's places, and
     //    the per-token exponent maximum (lanes holding the same token reduce
     //    in the warp: one shared-memory atomic per token and warp)
@@ -1047,6 +1059,58 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     }
     if (lo_used) atomicOr(&flags[0], 1u);
     named_bar(BAR_CONSUMERS, NCT);
+    } else {
+      // W4A4: X is quantised to NVFP4 here by the weights' quantiser steps,
+      // under the per-tensor scale gs_x = amax(|X|) / 2688 of this X (every
+      // CTA reads all of X for it, so all CTAs agree). B is the exact f16
+      // product e2m1(code) * e4m3(scale) of each element (the lo plane stays
+      // zero, the per-token factor is 1) and gs_x multiplies the sums.
+      uint32_t* amax_s = reinterpret_cast<uint32_t*>(misc + MISC_XAMAX);
+      const int per_tok = p.K / 8;
+      uint32_t mag = 0u;
+      for (int u = ctid; u < p.M * per_tok; u += NCT) {
+        const int m = u / per_tok;
+        mag = max(mag, bf16_mag_max8(*reinterpret_cast<const uint4*>(p.x + size_t(m) * p.K + 8 * (u - m * per_tok))));
+      }
+      mag = __reduce_max_sync(0xffffffffu, mag);
+      if ((ctid & 31) == 0) atomicMax(amax_s, mag);
+      named_bar(BAR_CONSUMERS, NCT);
+      const float gsx = __fdiv_rn(__uint_as_float(*amax_s << 16), 2688.0f);   // 6 * 448
+      // 16-element blocks of the staged K-steps: chunk pairs (2i, 2i+1) of a token
+      const int nbt = nx / 2;
+      for (int u = ctid; u < p.M * nbt; u += NCT) {
+        const int m = u / nbt, kc = chunk_of(2 * (u - m * nbt));
+        const uint16_t* src = p.x + size_t(m) * p.K + k0e + 8 * kc;
+        const uint4 xa = *reinterpret_cast<const uint4*>(src), xb = *reinterpret_cast<const uint4*>(src + 8);
+        const uint32_t wv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          v[2 * i] = __uint_as_float(wv[i] << 16);
+          v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+        }
+        uint32_t s_code, q[2];
+        quantize_block16(v, gsx, s_code, q);
+        const uint32_t sc = bcast_lo(e4m3x2_to_f16x2(s_code));
+        uint32_t h[8];
+        e2m1x8_to_f16x2x4(q[0], h);
+        e2m1x8_to_f16x2x4(q[1], h + 4);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = hmul2(h[i], sc);   // exact products
+        uint8_t* ch = sX + size_t(m) * p.xstride;
+        uint8_t* cl = sX + size_t(p.M + m) * p.xstride;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          *reinterpret_cast<uint2*>(ch + x_off(8 * kc + 4 * c)) = make_uint2(h[2 * c], h[2 * c + 1]);
+          *reinterpret_cast<uint2*>(cl + x_off(8 * kc + 4 * c)) = make_uint2(0u, 0u);
+        }
+      }
+      if (ctid == 0) {
+        *reinterpret_cast<float*>(misc + MISC_XGS) = gsx;
+        for (int m = 0; m < p.M; ++m) emax[m] = 14;
+      }
+      named_bar(BAR_CONSUMERS, NCT);
+    }
     const bool need_lo = flags[0] != 0u;
 
     if constexpr (MC == 1) {
@@ -1145,6 +1209,7 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   // From XR_MIN_M: 2M columns would force several K-slices; X goes through
   // the ring.
   c.xr = c.M >= XR_MIN_M;
+  if (c.act4 && c.xr) return cudaErrorInvalidConfiguration;   // W4A4: staged X only
   int S = 1;
   if (c.xr) {
     c.x_box = 4 * XGROUP_BYTES;
@@ -1236,7 +1301,7 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
   Params p;
   p.M = c.M; p.N = c.N; p.K = c.K; p.tiles = c.tiles; p.S = c.S; p.P = c.P;
   p.ks_base = c.ks_base; p.ks_rem = c.ks_rem; p.ncols = c.ncols; p.xk_max = c.xk_max;
-  p.xstride = c.xstride; p.pmax = c.pmax; p.nstage = c.nstage; p.tpc = c.tpc;
+  p.xstride = c.xstride; p.pmax = c.pmax; p.nstage = c.nstage; p.tpc = c.tpc; p.act4 = c.act4;
   p.xbytes = c.xbytes; p.xbox_words = c.x_box / 4; p.xbox_bytes = c.ncols * c.x_box;
   p.gs = gs; p.x = x; p.y = y;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);

@@ -62,6 +62,7 @@ struct MmaConfig {
   int epi;   // 0: Y; 1: SiLU-gated pairs of rows; 2: per-token argmax (k_mma.cu)
   int tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, nstage, grid;
   int tpc;   // whole tiles per CTA (no split tiles), 0: stream-K
+  int act4;  // W4A4: X quantised to NVFP4 inside the kernel (staged X only)
   bool split;
   // X in the ring (M > 4): X planes prepared once per call in the workspace
   bool xr;

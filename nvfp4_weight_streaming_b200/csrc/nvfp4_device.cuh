@@ -83,6 +83,53 @@ __device__ __forceinline__ uint32_t ld_stream_u16(const void* p) {
   return r;
 }
 
+// E4M3 round-to-nearest-even with saturation (hardware conversion); the
+// result's low byte is the code of `u`.
+__device__ __forceinline__ uint32_t e4m3_rne_sat(float u) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(u));
+  return r & 0xFFu;
+}
+
+// Two E2M1 codes (RNE, saturating): `lo` in bits 0..3, `hi` in bits 4..7.
+// A code of magnitude 0 is stored as 0x0 (no negative zero).
+__device__ __forceinline__ uint32_t e2m1x2_rne_sat(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r) : "f"(hi), "f"(lo));
+  if ((r & 0x07u) == 0) r &= 0xF0u;
+  if ((r & 0x70u) == 0) r &= 0x0Fu;
+  return r;
+}
+
+
+// One 16-element block of the NVFP4 quantiser under the per-tensor scale gs:
+// s = E4M3_RNE_satfinite((amax_b / 6) / gs), codes = E2M1_RNE_satfinite(v /
+// (e4m3(s) * gs)), each an fp32 operation in that order (all codes zero when
+// e4m3(s) * gs is 0). packed: element 2j in the low nibble of byte j.
+__device__ __forceinline__ void quantize_block16(const float v[16], float gs, uint32_t& s_code,
+                                                 uint32_t packed[2]) {
+  float amax_b = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax_b = fmaxf(amax_b, fabsf(v[i]));
+  const float t = __fdiv_rn(amax_b, 6.0f);
+  const float u = (gs > 0.0f) ? __fdiv_rn(t, gs) : 0.0f;
+  s_code = e4m3_rne_sat(u);
+  const float ds = __half2float(__ushort_as_half(
+      static_cast<unsigned short>(e4m3x2_to_f16x2(s_code) & 0xFFFFu)));
+  const float denom = __fmul_rn(ds, gs);
+  packed[0] = packed[1] = 0u;
+  if (denom > 0.0f) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t byte = e2m1x2_rne_sat(__fdiv_rn(v[2 * j], denom), __fdiv_rn(v[2 * j + 1], denom));
+      packed[j / 4] |= byte << (8 * (j % 4));
+    }
+  }
+}
+
 // ---- shared memory barriers and TMA ----------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
