@@ -39,8 +39,12 @@
  * variant (GEMV) has no such range condition.
  *
  * Conventions.
- *   - Every buffer is device memory owned by the caller; the library never
- *     allocates device memory. A plan holds only launch parameters.
+ *   - Every buffer is device memory owned by the caller; the library makes
+ *     no device allocation at run time. It holds one fixed array of
+ *     NVFP4_STATIC_SCRATCH_BYTES per device where its device code is loaded
+ *     (a __device__ variable, reserved when the module loads), used only by
+ *     nvfp4_linear_run_static. A plan holds only launch parameters and
+ *     cached TMA descriptors.
  *   - Calls that take a stream are asynchronous on it (a cudaStream_t passed
  *     as void*; NULL = legacy default stream), except nvfp4_linear_status,
  *     which synchronises that stream.
@@ -72,7 +76,7 @@ typedef enum {
   NVFP4_ERR_MISALIGNED = 3,    /* a pointer breaks the alignment rule */
   NVFP4_ERR_CUDA = 4,          /* a CUDA runtime call failed */
   NVFP4_ERR_TIMEOUT = 5,       /* a bounded device wait gave up (status word) */
-  NVFP4_ERR_BAD_SCALE = 6,     /* reserved: scale/global checks report counts */
+  NVFP4_ERR_BAD_SCALE = 6,     /* reserved, never returned: the scale checks report counts */
   NVFP4_ERR_WORKSPACE = 7      /* workspace missing or smaller than required */
 } nvfp4_status;
 
@@ -218,7 +222,10 @@ nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
  *     unspecified). NULL skips the copy.
  *   - The first call on a device looks up the array's address with that
  *     device current, which may load the library's device code there; make
- *     that first call before any stream capture.
+ *     that first call before any stream capture. The address is kept for
+ *     the life of the process: after a cudaDeviceReset (or anything else
+ *     that destroys the device's primary context) it is stale, and this
+ *     entry point must not be called again on that device.
  *   - Every call on a device shares the one array and leaves the last call's
  *     contents in it; each call clears, on `stream`, the part that must start
  *     at zero (status word and counters). Calls on one stream are therefore
