@@ -364,9 +364,11 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
 __global__ void __launch_bounds__(256)
 k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ planes, int pitch,
         int* __restrict__ emax_out, uint32_t* __restrict__ lo_out) {
-  // X may be the previous grid's output; the main kernel may start now
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The main kernel may launch now (it waits for this grid before it reads
+  // the planes, and meanwhile streams weights); X may be the previous grid's
+  // output.
   if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ int s_max[8];
   const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint4* row = reinterpret_cast<const uint4*>(x + size_t(m) * K);
