@@ -118,6 +118,10 @@ bool lookup_maps(nvfp4_plan_s* p, const void* wp, const void* ws, CUtensorMap* m
   if (p->variant == int(NVFP4_VARIANT_ROW)) {
     ok = nvfp4::encode_row_maps(p->N, p->K, p->row.ipu, p->row.fmt, static_cast<const uint8_t*>(wp),
                                 static_cast<const uint8_t*>(ws), &e.mw, &e.ms);
+  } else if (p->variant == int(NVFP4_VARIANT_MMA) && p->fmt == 1) {
+    // FP8 codes; the row scales are read directly (the second map is unused)
+    ok = nvfp4::encode_fp8_codes_map(p->N, p->K, static_cast<const uint8_t*>(wp), &e.mw);
+    e.ms = e.mw;
   } else {
     const int box_rows = p->variant == int(NVFP4_VARIANT_MMA) ? nvfp4::kMmaTileRows : 128;
     ok = nvfp4::encode_weight_maps(p->N, p->K, box_rows, static_cast<const uint8_t*>(wp),
@@ -191,7 +195,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   p.ws_bytes = 0;
   unsigned forced = flags & NVFP4_PLAN_VARIANT_MASK;
   p.variant = forced ? int(forced)
-                     : (fmt == 1 ? int(NVFP4_VARIANT_ROW) : act4 ? int(NVFP4_VARIANT_MMA) : auto_variant(M, N, K));
+                     : (fmt == 1 || act4 ? int(NVFP4_VARIANT_MMA) : auto_variant(M, N, K));
   if (K == 0 || N == 0) {
     // nothing to contract: run() writes zeros (K == 0) or returns (N == 0)
     if (p.variant == int(NVFP4_VARIANT_GEMV) && M > 4) p.variant = int(NVFP4_VARIANT_TC);
@@ -199,7 +203,9 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   auto configure = [&]() -> nvfp4_status {
     nvfp4_status st = NVFP4_OK;
     if (p.epi != 0 && p.variant != int(NVFP4_VARIANT_MMA)) return NVFP4_ERR_UNSUPPORTED;
-    if (p.fmt != 0 && (p.variant != int(NVFP4_VARIANT_ROW) || p.epi != 0)) return NVFP4_ERR_UNSUPPORTED;
+    if (p.fmt != 0 && ((p.variant != int(NVFP4_VARIANT_ROW) && p.variant != int(NVFP4_VARIANT_MMA)) ||
+                       p.epi != 0 || p.act4 != 0))
+      return NVFP4_ERR_UNSUPPORTED;
     if (p.act4 && p.variant != int(NVFP4_VARIANT_MMA)) return NVFP4_ERR_UNSUPPORTED;
     switch (p.variant) {
       case NVFP4_VARIANT_GEMV: {
@@ -210,7 +216,7 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
       }
       case NVFP4_VARIANT_MMA: {
         if (K == 0 || N == 0) break;
-        p.mma.M = M; p.mma.N = N; p.mma.K = K; p.mma.epi = p.epi; p.mma.act4 = p.act4;
+        p.mma.M = M; p.mma.N = N; p.mma.K = K; p.mma.epi = p.epi; p.mma.act4 = p.act4; p.mma.fmt = p.fmt;
         cudaError_t e = nvfp4::mma_configure(p.mma, sms);
         if (e == cudaSuccess && !nvfp4::tensor_maps_supported()) e = cudaErrorNotSupported;
         if (e == cudaErrorInvalidConfiguration || e == cudaErrorNotSupported) st = NVFP4_ERR_UNSUPPORTED;
@@ -246,6 +252,13 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
     return st;
   };
   nvfp4_status st = configure();
+  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.fmt == 1 && p.variant == int(NVFP4_VARIANT_MMA)) {
+    // FP8 weights the MMA variant cannot take (X does not fit beside its ring): the row variant
+    p.variant = int(NVFP4_VARIANT_ROW);
+    p.split_k = 1;
+    p.ws_bytes = 0;
+    st = configure();
+  }
   if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.fmt == 0 && p.variant != int(NVFP4_VARIANT_MMA) &&
       p.variant != int(NVFP4_VARIANT_TC)) {
     // the table's choice (GEMV, row) cannot take this shape or epilogue
@@ -335,7 +348,8 @@ nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
           }
           mx = plan->xmap;
         }
-        e = nvfp4::launch_mma(plan->mma, &mw, &ms, &mx, w_global, xb, yb, workspace,
+        const float* row_scale = plan->fmt == 1 ? static_cast<const float*>(static_cast<const void*>(w_scales)) : nullptr;
+        e = nvfp4::launch_mma(plan->mma, &mw, &ms, &mx, w_global, row_scale, xb, yb, workspace,
                               stall ? kStallTimeoutCycles : kTimeoutCycles, stall, pdl, st);
         break;
       }

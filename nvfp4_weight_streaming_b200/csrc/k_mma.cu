@@ -77,6 +77,12 @@ constexpr int NSTAGE_MAX = 8;             // deeper rings use what X leaves free
 constexpr int W_BYTES = TROWS * KS / 2;    // 32768
 constexpr int S_BYTES = TROWS * KS / 16;   // 4096
 constexpr int STAGE_BYTES = W_BYTES + S_BYTES;
+// FP8 weight tier: E4M3 codes [N][K], one fp32 scale per row; a stage holds
+// 256 rows x 256 codes as two 128-byte-wide swizzled halves (K 0..127, 128..255)
+constexpr int FMT_NVFP4 = 0, FMT_FP8 = 1;
+constexpr int W_BYTES_FP8 = TROWS * KS;    // 65536
+__host__ __device__ constexpr int w_bytes_of(int fmt) { return fmt == FMT_FP8 ? W_BYTES_FP8 : W_BYTES; }
+__host__ __device__ constexpr int s_bytes_of(int fmt) { return fmt == FMT_FP8 ? 0 : S_BYTES; }
 constexpr int MISC_BASE = 1024;            // barriers, flags, lists
 // misc area size: for M <= 4 plus the prefetched piece [M][TROWS] floats
 inline int misc_bytes(int M) { return MISC_BASE + (M <= 4 ? M * TROWS * 4 : 0); }
@@ -98,6 +104,7 @@ struct Params {
   int M, N, K, tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, nstage;
   int tpc;                                   // whole tiles per CTA (no split tiles), 0: stream-K
   int act4;                                  // W4A4: X quantised to NVFP4 in the kernel
+  const float* row_scale;                    // FP8 tier: fp32 scale of each weight row [N]
   int xbytes, xbox_words, xbox_bytes;        // X in the ring: stage area, words per column, box bytes
   const int* xemax;                          // X in the ring: per-token exponent maximum
   const uint32_t* xlo;                       // X in the ring: per-token "lo plane used"
@@ -512,12 +519,46 @@ __device__ __forceinline__ void compute_step_bd(const uint8_t* sw, const uint8_t
   }
 }
 
+// FP8 step: the same K mapping as compute_step (lane quad t holds elements
+// 64t..64t+63 of rows r and r+8, MMA i takes 64t + 4i + {0..3}), on E4M3
+// codes: one cvt.rn.f16x2.e4m3x2 per pair of codes is the exact A fragment
+// (the row scale is applied to the finished sums). Elements 64t.. sit in
+// half t >> 1 of the stage, 16-byte chunks 4 (t & 1) .. 4 (t & 1) + 3.
+template <int NTILE, bool PRED>
+__device__ __forceinline__ void compute_step_fp8(const uint8_t* sw, int r, float (*acc)[4], const uint8_t* sx,
+                                                 const uint32_t* xcol, const bool* xon, uint32_t xg, int t) {
+  const int r1 = r + 8;
+  const uint8_t* hb = sw + (t >> 1) * (TROWS * 128);
+  const int cb = 4 * (t & 1);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 c0 = *reinterpret_cast<const uint4*>(hb + r * 128 + (((cb + j) ^ (r & 7)) << 4));
+    const uint4 c1 = *reinterpret_cast<const uint4*>(hb + r1 * 128 + (((cb + j) ^ (r1 & 7)) << 4));
+    const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w}, w1[4] = {c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int i = 4 * j + q;
+      const uint32_t a0 = e4m3x2_to_f16x2(w0[q]);         // row r,   k = 4i, 4i+1
+      const uint32_t a1 = e4m3x2_to_f16x2(w1[q]);         // row r+8, k = 4i, 4i+1
+      const uint32_t a2 = e4m3x2_to_f16x2(w0[q] >> 16);   // row r,   k = 4i+2, 4i+3
+      const uint32_t a3 = e4m3x2_to_f16x2(w1[q] >> 16);   // row r+8, k = 4i+2, 4i+3
+      constexpr int NSET = 4 / NTILE;
+#pragma unroll
+      for (int nt = 0; nt < NTILE; ++nt) {
+        uint2 bb = make_uint2(0u, 0u);
+        if (!PRED || xon[nt]) bb = *reinterpret_cast<const uint2*>(sx + (xcol[nt] + xg) + 8 * i);
+        mma16816(acc[(i % NSET) * NTILE + nt], a0, a1, a2, a3, bb.x, bb.y);
+      }
+    }
+  }
+}
+
 // Consumer warp's walk over the CTA's units. MC = token class (1: M <= 4,
 // 2: M <= 8, 3: M <= 16); NTILE token tiles per A fragment (1: hi and lo in
 // one tile; 2: hi + lo tiles, or two hi tiles; 4: two hi + two lo tiles).
 // Pieces of split tiles are written to the workspace and handed to the
 // settler warp through the queue (mbarriers q_full / q_empty).
-template <int MC, int NTILE, bool LO, bool XR, int EPI>
+template <int MC, int NTILE, bool LO, bool XR, int EPI, int FMT>
 __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* sS, const uint8_t* sX,
                                         const int* emax, uint32_t b_full, uint32_t b_empty,
                                         uint32_t b_qfull, uint32_t b_qempty,
@@ -576,7 +617,9 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
     constexpr bool EARLY = false;
     // lane t reads 64-element group t of this step (staged X: of the slice)
     const uint32_t xg = uint32_t(XGROUP_BYTES * (XR ? t : 4 * j + t));
-    if constexpr (MC == 0)
+    if constexpr (FMT == FMT_FP8)
+      compute_step_fp8<NTILE, LO>(sW + st * W_BYTES_FP8, r, acc, XR ? sX + st * p.xbytes : sX, xcol, xon, xg, t);
+    else if constexpr (MC == 0)
       compute_step_bd(sW + st * W_BYTES, sS + st * S_BYTES, r, acc, (XR ? sX + st * p.xbytes : sX) + xcol[0],
                       xon[0], xg, t);
     else
@@ -672,6 +715,16 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
         v[e][1] = at[0][2 + e] * fh[e] + l1 * fl[e];
         v[2 + e][0] = at[1 % NTILE][e] * fh[2 + e] + l2 * fl[2 + e];
         v[2 + e][1] = at[1 % NTILE][2 + e] * fh[2 + e] + l3 * fl[2 + e];
+      }
+    }
+    if constexpr (FMT == FMT_FP8) {
+      // the rows' fp32 scales (rows past N read nothing)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int n = tcur * TROWS + r + 8 * h;
+        const float rs = n < p.N ? __ldg(p.row_scale + n) : 0.0f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e][h] *= rs;
       }
     }
     if (p.act4) {
@@ -864,7 +917,7 @@ __device__ __forceinline__ void settle(const Params& p, uint32_t b_qfull, uint32
 // XR: X in the ring. Each stage also carries one K-step of the X planes
 // (prepared by k_xprep in the workspace), there are no K-slices and no
 // staging; otherwise the CTA stages its K-slice of X in shared memory.
-template <int MC, bool XR, int EPI>
+template <int MC, bool XR, int EPI, int FMT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
       const __grid_constant__ CUtensorMap tm_x, const Params p) {
@@ -875,8 +928,8 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int nst = p.nstage;
   uint8_t* sW = smem;                                     // nst x 32 KB (1024-aligned)
-  uint8_t* sS = smem + nst * W_BYTES;                     // nst x 4 KB
-  uint8_t* sX = sS + nst * S_BYTES;                       // staged slice, or nst X boxes
+  uint8_t* sS = smem + nst * w_bytes_of(FMT);             // nst x 4 KB (NVFP4; none for FP8)
+  uint8_t* sX = sS + nst * s_bytes_of(FMT);               // staged slice, or nst X boxes
   uint8_t* misc = sX + (XR ? size_t(nst) * p.xbytes : size_t(p.ncols) * p.xstride);
   uint64_t* bars = reinterpret_cast<uint64_t*>(misc);     // full[8] empty[8] qfull[8] qempty[8]
   int* emax = reinterpret_cast<int*>(misc + MISC_EMAX);   // [16]
@@ -940,11 +993,19 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
           }
           if (!wait_bar(b_empty + 8 * st, ph ^ 1u, abort_flag, p, ST_TIMEOUT_PRODUCER)) break;
           // the X box delivers exactly xbox_bytes (2M columns of one K-step)
-          mbar_expect_tx(b_full + 8 * st, STAGE_BYTES + (XR ? p.xbox_bytes : 0));
-          tma_load_2d_hint(smem_u32(sW + st * W_BYTES), &tm_w, (ks0 + j) * (KS / 2), tile * TROWS,
-                           b_full + 8 * st, pol);
-          tma_load_2d_hint(smem_u32(sS + st * S_BYTES), &tm_s, (ks0 + j) * (KS / 16), tile * TROWS,
-                           b_full + 8 * st, pol);
+          mbar_expect_tx(b_full + 8 * st, w_bytes_of(FMT) + s_bytes_of(FMT) + (XR ? p.xbox_bytes : 0));
+          if constexpr (FMT == FMT_FP8) {
+            // two 128-byte-wide halves of the 256 codes of each row
+            tma_load_2d_hint(smem_u32(sW + st * W_BYTES_FP8), &tm_w, (ks0 + j) * KS, tile * TROWS,
+                             b_full + 8 * st, pol);
+            tma_load_2d_hint(smem_u32(sW + st * W_BYTES_FP8 + TROWS * 128), &tm_w, (ks0 + j) * KS + 128,
+                             tile * TROWS, b_full + 8 * st, pol);
+          } else {
+            tma_load_2d_hint(smem_u32(sW + st * W_BYTES), &tm_w, (ks0 + j) * (KS / 2), tile * TROWS,
+                             b_full + 8 * st, pol);
+            tma_load_2d_hint(smem_u32(sS + st * S_BYTES), &tm_s, (ks0 + j) * (KS / 16), tile * TROWS,
+                             b_full + 8 * st, pol);
+          }
           if (XR && x_first)
             tma_load_2d(smem_u32(sX + st * p.xbytes), &tm_x, (ks0 + j) * p.xbox_words, 0, b_full + 8 * st);
           if (++j == cnt) { j = 0; ++tile; }
@@ -979,13 +1040,13 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const int cw = warp - 1;
 #define NVFP4_CONSUME(MC_, NT_, LO_, XR_, EMAX_) \
-  consume<MC_, NT_, LO_, XR_, EPI>(p, sW, sS, sX, EMAX_, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, pre_flag, pre_buf, s, cnt, a, b, L, cw, lane)
+  consume<MC_, NT_, LO_, XR_, EPI, FMT>(p, sW, sS, sX, EMAX_, b_full, b_empty, b_qfull, b_qempty, abort_flag, skip, pre_flag, pre_buf, s, cnt, a, b, L, cw, lane)
     if constexpr (XR) {
       // X arrives with the weights; exponents and lo flags come from k_xprep
       bool need_lo = false;
       for (int m = 0; m < p.M; ++m) need_lo |= p.xlo[m] != 0u;
       if constexpr (MC == 1) {
-        if (p.M == 1 || (p.M == 2 && !need_lo)) NVFP4_CONSUME(0, 1, false, true, p.xemax);
+        if (FMT == FMT_NVFP4 && (p.M == 1 || (p.M == 2 && !need_lo))) NVFP4_CONSUME(0, 1, false, true, p.xemax);
         else if (need_lo) NVFP4_CONSUME(1, 1, true, true, p.xemax); else NVFP4_CONSUME(1, 1, false, true, p.xemax);
       } else if constexpr (MC == 2) {
         if (need_lo) NVFP4_CONSUME(2, 2, true, true, p.xemax); else NVFP4_CONSUME(2, 1, false, true, p.xemax);
@@ -1116,7 +1177,7 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     const bool need_lo = flags[0] != 0u;
 
     if constexpr (MC == 1) {
-      if (p.M == 1 || (p.M == 2 && !need_lo)) NVFP4_CONSUME(0, 1, false, false, emax);
+      if (FMT == FMT_NVFP4 && (p.M == 1 || (p.M == 2 && !need_lo))) NVFP4_CONSUME(0, 1, false, false, emax);
       else if (need_lo) NVFP4_CONSUME(1, 1, true, false, emax); else NVFP4_CONSUME(1, 1, false, false, emax);
     } else if constexpr (MC == 2) {
       if (need_lo) NVFP4_CONSUME(2, 2, true, false, emax); else NVFP4_CONSUME(2, 1, false, false, emax);
@@ -1168,10 +1229,12 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
 template <int EPI>
 cudaError_t set_smem_attrs(int optin) {
   using namespace mm;
-  cudaError_t e = cudaFuncSetAttribute(k_mma<1, false, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<1, true, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<2, true, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<3, true, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  cudaError_t e = cudaFuncSetAttribute(k_mma<1, false, EPI, FMT_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<1, true, EPI, FMT_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<2, true, EPI, FMT_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<3, true, EPI, FMT_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess && EPI == EPI_NONE)
+    e = cudaFuncSetAttribute(k_mma<1, false, EPI_NONE, FMT_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   return e;
 }
 
@@ -1180,12 +1243,13 @@ template <int EPI>
 cudaError_t launch_main(const MmaConfig& c, cudaLaunchConfig_t* cfg, const CUtensorMap& mw, const CUtensorMap& ms,
                         const CUtensorMap& mx, const mm::Params& p) {
   using namespace mm;
+  if (c.fmt == FMT_FP8) return cudaLaunchKernelEx(cfg, k_mma<1, false, EPI_NONE, FMT_FP8>, mw, ms, mx, p);
   if (c.M <= 4) {
-    if (c.xr) return cudaLaunchKernelEx(cfg, k_mma<1, true, EPI>, mw, ms, mx, p);
-    return cudaLaunchKernelEx(cfg, k_mma<1, false, EPI>, mw, ms, mx, p);
+    if (c.xr) return cudaLaunchKernelEx(cfg, k_mma<1, true, EPI, FMT_NVFP4>, mw, ms, mx, p);
+    return cudaLaunchKernelEx(cfg, k_mma<1, false, EPI, FMT_NVFP4>, mw, ms, mx, p);
   }
-  if (c.M <= 8) return cudaLaunchKernelEx(cfg, k_mma<2, true, EPI>, mw, ms, mx, p);
-  return cudaLaunchKernelEx(cfg, k_mma<3, true, EPI>, mw, ms, mx, p);
+  if (c.M <= 8) return cudaLaunchKernelEx(cfg, k_mma<2, true, EPI, FMT_NVFP4>, mw, ms, mx, p);
+  return cudaLaunchKernelEx(cfg, k_mma<3, true, EPI, FMT_NVFP4>, mw, ms, mx, p);
 }
 
 cudaError_t mma_configure(MmaConfig& c, int num_sms) {
@@ -1212,13 +1276,16 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   // the ring.
   c.xr = c.M >= XR_MIN_M;
   if (c.act4 && c.xr) return cudaErrorInvalidConfiguration;   // W4A4: staged X only
+  // FP8 weights: staged X, no epilogue, no W4A4 (a 64 KB stage leaves no room for X boxes)
+  if (c.fmt == FMT_FP8 && (c.xr || c.epi != EPI_NONE || c.act4)) return cudaErrorInvalidConfiguration;
+  const int stage_bytes = w_bytes_of(c.fmt) + s_bytes_of(c.fmt);
   int S = 1;
   if (c.xr) {
     c.x_box = 4 * XGROUP_BYTES;
     c.x_pitch = (c.K / 64) * XGROUP_BYTES;
     c.xbytes = ((c.ncols * c.x_box + 127) / 128) * 128;
   } else {
-    const long long x_budget = (long long)optin - 1024 - (long long)NSTAGE_MIN * STAGE_BYTES - misc_bytes(c.M);
+    const long long x_budget = (long long)optin - 1024 - (long long)NSTAGE_MIN * stage_bytes - misc_bytes(c.M);
     auto fits = [&](int ks) { return (long long)c.ncols * stride_for(ks) <= x_budget; };
     if (!fits(1)) return cudaErrorInvalidConfiguration;
     int max_ks = 1;
@@ -1267,11 +1334,11 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   {
     const long long x_smem = c.xr ? 0 : (long long)c.ncols * c.xstride;
     const long long left = (long long)optin - 1024 - x_smem - misc_bytes(c.M);
-    int nst = int(left / (STAGE_BYTES + c.xbytes));
+    int nst = int(left / (stage_bytes + c.xbytes));
     c.nstage = nst < NSTAGE_MAX ? nst : NSTAGE_MAX;
   }
   if (c.nstage < NSTAGE_MIN) return cudaErrorInvalidConfiguration;
-  c.smem = 1024 + size_t(c.nstage) * (STAGE_BYTES + c.xbytes) +
+  c.smem = 1024 + size_t(c.nstage) * (stage_bytes + c.xbytes) +
            (c.xr ? 0 : size_t(c.ncols) * c.xstride) + misc_bytes(c.M);
   if (c.smem > size_t(optin)) return cudaErrorInvalidConfiguration;
   // workspace: status word, per-(tile, row group) counters, partial sums,
@@ -1296,16 +1363,30 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   return e;
 }
 
+// FP8 weight tier: the E4M3 codes [N][K] as boxes of 128 bytes x 256 rows
+// with the 128-byte swizzle (two per 256-code K-step).
+bool encode_fp8_codes_map(int N, int K, const uint8_t* wp, void* map_w) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dim[2] = {cuuint64_t(K), cuuint64_t(N)};
+  const cuuint64_t str[1] = {cuuint64_t(K)};
+  const cuuint32_t box[2] = {128, cuuint32_t(mm::TROWS)};
+  const cuuint32_t one[2] = {1, 1};
+  return fn(static_cast<CUtensorMap*>(map_w), CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(wp), dim, str,
+            box, one, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s, const void* map_x,
-                       const float* gs, const uint16_t* x, uint16_t* y, void* workspace,
-                       long long timeout_cycles, bool stall, bool pdl, cudaStream_t st) {
+                       const float* gs, const float* row_scale, const uint16_t* x, uint16_t* y,
+                       void* workspace, long long timeout_cycles, bool stall, bool pdl, cudaStream_t st) {
   using namespace mm;
   Params p;
   p.M = c.M; p.N = c.N; p.K = c.K; p.tiles = c.tiles; p.S = c.S; p.P = c.P;
   p.ks_base = c.ks_base; p.ks_rem = c.ks_rem; p.ncols = c.ncols; p.xk_max = c.xk_max;
   p.xstride = c.xstride; p.pmax = c.pmax; p.nstage = c.nstage; p.tpc = c.tpc; p.act4 = c.act4;
   p.xbytes = c.xbytes; p.xbox_words = c.x_box / 4; p.xbox_bytes = c.ncols * c.x_box;
-  p.gs = gs; p.x = x; p.y = y;
+  p.gs = gs; p.x = x; p.y = y; p.row_scale = row_scale;
   uint8_t* wsb = static_cast<uint8_t*>(workspace);
   p.status = reinterpret_cast<uint32_t*>(wsb);
   p.counters = reinterpret_cast<uint32_t*>(wsb + c.ws_counters_off);

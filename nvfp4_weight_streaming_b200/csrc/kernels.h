@@ -63,6 +63,7 @@ struct MmaConfig {
   int tiles, S, P, ks_base, ks_rem, ncols, xk_max, xstride, pmax, nstage, grid;
   int tpc;   // whole tiles per CTA (no split tiles), 0: stream-K
   int act4;  // W4A4: X quantised to NVFP4 inside the kernel (staged X only)
+  int fmt;   // 0: NVFP4 weights; 1: FP8 weights (E4M3 codes [N][K], fp32 row scales [N]; M <= 4, staged X)
   bool split;
   // X in the ring (M > 4): X planes prepared once per call in the workspace
   bool xr;
@@ -73,8 +74,10 @@ struct MmaConfig {
 cudaError_t mma_configure(MmaConfig& c, int num_sms);
 // map_x: descriptor of the X planes in `workspace` (encode_x_planes_map), used when c.xr.
 cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s, const void* map_x,
-                       const float* gs, const uint16_t* x, uint16_t* y, void* workspace,
-                       long long timeout_cycles, bool stall, bool pdl, cudaStream_t st);
+                       const float* gs, const float* row_scale, const uint16_t* x, uint16_t* y,
+                       void* workspace, long long timeout_cycles, bool stall, bool pdl, cudaStream_t st);
+// FP8 weight tier codes map for the MMA variant.
+bool encode_fp8_codes_map(int N, int K, const uint8_t* wp, void* map_w);
 constexpr int kMmaTileRows = 256;
 
 // The driver's cuTensorMapEncodeTiled (null if unavailable); k_tc.cu.

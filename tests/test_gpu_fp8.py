@@ -4,7 +4,8 @@ The tier stores W as E4M3 codes [N][K] with one fp32 scale per row (reading
 R15: s_n = amax|W[n]| / 448, code = E4M3_RNE_satfinite(w / s_n)); the GPU
 quantiser must reproduce the oracle's codes and scales bit for bit, and the
 linear must meet the stated tolerance against the oracle's fp64 sum of
-e4m3(code) * s_n * x. Runs on the row-block variant (M <= 2).
+e4m3(code) * s_n * x. Runs on the MMA variant (the default, M <= 4) and on the
+row-block variant (forced, M <= 2).
 """
 import numpy as np
 import pytest
@@ -59,12 +60,12 @@ def test_fp8_quantizer_flags_nonfinite():
     assert gpu_quantize_fp8(W)[2] == 2
 
 
-def run_fp8(codes, sc, X, gs=1.0, repeat=1):
+def run_fp8(codes, sc, X, gs=1.0, repeat=1, variant=0):
     M, K = X.shape
     N = codes.shape[0]
-    plan = nv.nvfp4_linear_plan(M, N, K, torch.cuda.current_device(), nv.NVFP4_PLAN_WEIGHT_FP8)
+    plan = nv.nvfp4_linear_plan(M, N, K, torch.cuda.current_device(), nv.NVFP4_PLAN_WEIGHT_FP8 | variant)
     try:
-        assert nv.nvfp4_linear_variant(plan) == nv.NVFP4_VARIANT_ROW
+        assert nv.nvfp4_linear_variant(plan) == (variant or nv.NVFP4_VARIANT_MMA)
         wsb = nv.nvfp4_linear_workspace_bytes(plan)
         ws = torch.zeros(max(wsb, 16), dtype=torch.uint8, device="cuda")
         cd = torch.from_numpy(codes).cuda()
@@ -82,14 +83,35 @@ def run_fp8(codes, sc, X, gs=1.0, repeat=1):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 520, 512), (2, 1000, 768), (1, 2, 256), (2, 2339, 5120),
-                                   (1, 34816, 5120), (1, 5120, 17408)])
-def test_fp8_linear(M, N, K):
+                                   (1, 34816, 5120), (1, 5120, 17408), (3, 777, 1280),
+                                   (4, 130 * 256 - 77, 512)])
+@pytest.mark.parametrize("variant", [0, nv.NVFP4_VARIANT_ROW])
+def test_fp8_linear(M, N, K, variant):
+    if variant == nv.NVFP4_VARIANT_ROW and M > 2:
+        pytest.skip("the row variant takes M <= 2")
     W = synth.normal_f32(N * K, 0.02, seed=N + K, stream=7).reshape(N, K)
     codes, sc = oracle.quantize_fp8_rows(W)
     X = synth.x_bf16_custom(synth.X_OUTLIERS, M, K, seed=K, n_outliers=8, gain=20.0)
-    y = run_fp8(codes, sc, X)
+    y = run_fp8(codes, sc, X, variant=variant)
     y_ref, ad = oracle.linear_fp8(codes, sc, X, M, N, K)
     check_tolerance(y, y_ref, ad)
+
+
+def test_fp8_dyadic_case_is_exact_on_both_variants():
+    """Integer weights |v| <= 8 (exact E4M3 codes, from torch's conversion),
+    unit row scales and integer X: every partial sum is an exact integer in
+    fp32, so both variants must return the oracle's value rounded to bf16."""
+    M, N, K = 2, 300, 512
+    rng = np.random.default_rng(11)
+    vals = rng.integers(-8, 9, size=(N, K)).astype(np.float32)
+    codes = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    sc = np.ones(N, np.float32)
+    X = oracle.bf16_round_array(rng.integers(-4, 5, size=(M, K)).astype(np.float64))
+    y_ref, _ = oracle.linear_fp8(codes, sc, X, M, N, K)
+    want = oracle.bf16_bits_to_f64(oracle.bf16_round_array(y_ref))
+    for variant in (0, nv.NVFP4_VARIANT_ROW):
+        got = oracle.bf16_bits_to_f64(run_fp8(codes, sc, X, variant=variant))
+        assert np.array_equal(got, want), variant
 
 
 def test_fp8_linear_global_scale_multiplies():
@@ -132,12 +154,19 @@ def test_fp8_deterministic():
 
 def test_fp8_plan_limits():
     d = torch.cuda.current_device()
-    for flags in (nv.NVFP4_PLAN_WEIGHT_FP8 | nv.NVFP4_VARIANT_MMA,
+    for flags in (nv.NVFP4_PLAN_WEIGHT_FP8 | nv.NVFP4_VARIANT_GEMV,
                   nv.NVFP4_PLAN_WEIGHT_FP8 | nv.NVFP4_VARIANT_TC,
-                  nv.NVFP4_PLAN_WEIGHT_FP8 | nv.NVFP4_PLAN_EPI_SWIGLU):
+                  nv.NVFP4_PLAN_WEIGHT_FP8 | nv.NVFP4_PLAN_EPI_SWIGLU,
+                  nv.NVFP4_PLAN_WEIGHT_FP8 | nv.NVFP4_PLAN_ACT_NVFP4):
         with pytest.raises(nv.Nvfp4Error) as e:
             nv.nvfp4_linear_plan(1, 1024, 512, d, flags)
         assert e.value.status == nv.NVFP4_ERR_UNSUPPORTED
-    with pytest.raises(nv.Nvfp4Error) as e:
-        nv.nvfp4_linear_plan(3, 1024, 512, d, nv.NVFP4_PLAN_WEIGHT_FP8)
-    assert e.value.status == nv.NVFP4_ERR_UNSUPPORTED
+    for M, flags in ((5, 0), (3, nv.NVFP4_VARIANT_ROW)):
+        with pytest.raises(nv.Nvfp4Error) as e:
+            nv.nvfp4_linear_plan(M, 1024, 512, d, nv.NVFP4_PLAN_WEIGHT_FP8 | flags)
+        assert e.value.status == nv.NVFP4_ERR_UNSUPPORTED
+    p = nv.nvfp4_linear_plan(4, 1024, 512, d, nv.NVFP4_PLAN_WEIGHT_FP8)
+    try:
+        assert nv.nvfp4_linear_variant(p) == nv.NVFP4_VARIANT_MMA
+    finally:
+        nv.nvfp4_linear_destroy(p)
