@@ -22,7 +22,11 @@
 //                step maps its K slots to physical K as (2t, 2t+1) <-> 64t + 4i
 //                + {0, 1} and (2t+8, 2t+9) <-> 64t + 4i + {2, 3}, so every
 //                fragment is four consecutive elements of one lane. A warp
-//                releases a stage after its MMAs.
+//                releases a stage after its MMAs. For M = 1 (and M = 2 without
+//                a lo plane) the A fragments are the raw E2M1 values and the
+//                block scale is applied per 16-element block in fp32 instead
+//                (block-diagonal B, compute_step_bd). FP8 weights: the same K
+//                mapping on E4M3 codes, row scales applied to the sums.
 //   warp 17      settler: completes tiles split between CTAs (below).
 //
 // B is X in f16, scaled per token by a power of two (largest magnitude at
@@ -32,27 +36,32 @@
 // Columns are groups of 64 elements padded to 136 bytes, so B fragments are
 // bank-conflict-free 8-byte shared loads at immediate offsets. Every product
 // is exact; only the fp32 accumulation rounds. When no element needs the lo
-// plane, only hi tiles are issued. M <= 4: each CTA stages its K-slice of X in
-// shared memory. M >= 5 ("X in the ring"): k_xprep writes both planes once per
-// call into the workspace and every ring stage also carries one K-step box of
+// plane, only hi tiles are issued. M <= 4: each CTA stages the K-steps of X
+// its units touch in shared memory (W4A4: quantising them to NVFP4 on the
+// way). M >= 5 ("X in the ring"): k_xprep writes both planes once per call
+// into the workspace and every ring stage also carries one K-step box of
 // them, so these classes need no K-slices.
 //
-// Why not tcgen05 here: on B200 a tcgen05.mma kind::f16 with M = 128 costs ~85
-// cycles whatever N <= 128 is, i.e. at most 24 weight elements per clock per
-// SM, while this warp MMA sustains ~1000 MAC per clock per SM, i.e. 128
-// weight elements per clock at N = 8. For this skinny contraction the warp
-// MMA is the faster tensor path (the tcgen05 kernel is kept as variant TC).
+// Why not tcgen05 here: for N = 8..32 token columns a tcgen05.mma of M = 128
+// weight rows costs hundreds of cycles per instruction once its A operand
+// has to be decoded and stored by the warps (the variant TC kernel measures
+// ~400 SM cycles per MMA, tensor pipe 3% busy), while this warp MMA takes the
+// decoded fragments straight from registers at ~1000 MAC per clock per SM.
+// For this skinny contraction the warp MMA is the faster tensor path.
 //
-// Work split: K is cut into S slices (S = 1 unless a staged X slice would not
-// fit next to the ring); the CTAs of a slice share its (256-row tile, 256-k
-// step) units evenly (stream-K). Tiles a CTA covers entirely are stored
-// directly. A split tile is completed per 16-row group: the pieces write fp32
-// partials and count themselves on the group's counter; the last sums all
-// pieces in k order (results repeat bit for bit) and resets the counter. The
-// piece at the end of a CTA's range usually finds the tile's other piece
-// already counted and finishes the tile from its registers. Every mbarrier
-// wait is bounded; on expiry the CTA records the timeout in the workspace
-// status word, stops, drains its in-flight TMA loads and returns.
+// Work split: with at most as many 256-row tiles as SMs (and at least 85% of
+// them busy) every CTA takes one whole tile over all of K and stores it
+// directly: nothing crosses CTAs. Otherwise K is cut into S slices (S = 1
+// unless a staged X slice would not fit next to the ring) and the CTAs of a
+// slice share its (256-row tile, 256-k step) units evenly (stream-K). Tiles a
+// CTA covers entirely are stored directly. A split tile is completed per
+// 16-row group: the pieces write fp32 partials and count themselves on the
+// group's counter; the last sums all pieces in k order (results repeat bit
+// for bit) and resets the counter. The piece at the end of a CTA's range
+// usually finds the tile's other piece already counted and finishes the tile
+// from its registers. Every mbarrier wait is bounded; on expiry the CTA
+// records the timeout in the workspace status word, stops, drains its
+// in-flight TMA loads and returns.
 #include "kernels.h"
 #include "nvfp4_device.cuh"
 
