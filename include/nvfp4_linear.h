@@ -121,8 +121,7 @@ typedef struct nvfp4_plan_s* nvfp4_plan_t;
  * the tolerance and the X range are as for NVFP4. nvfp4_quantize_fp8 makes
  * such weights. */
 #define NVFP4_PLAN_WEIGHT_FP8 0x1000u
-/* W4A4 tier (plan flag; MMA variant with X staged in shared memory, i.e.
- * M <= 4, in K-slices where all of K does not fit): X arrives as bf16 like
+/* W4A4 tier (plan flag; MMA variant, any M): X arrives as bf16 like
  * always and is quantised to NVFP4 inside the kernel with the weights'
  * quantiser steps -- 16-element blocks of a token row, E4M3 block scales,
  * one per-tensor scale gs_x = amax(|X|) / (6 * 448) of the call's X (page
@@ -130,8 +129,9 @@ typedef struct nvfp4_plan_s* nvfp4_plan_t;
  * (NVIDIA ModelOpt)": weights and activations NVFP4). Y is then sum_k
  * w_hat[n][k] * x_hat[m][k] with x_hat = e2m1 * e4m3 * gs_x: a different
  * (quantised) result from the W4A16 linear; the same tolerance, against the
- * fp64 sum of w_hat * x_hat, applies. Plans that cannot stage X return
- * UNSUPPORTED, as do other variants and the FP8 weight tier. */
+ * fp64 sum of w_hat * x_hat, applies. For M <= 4 every CTA quantises the
+ * K-steps it stages; from M = 5 the X-conversion kernel quantises X once per
+ * call. Other variants and the FP8 weight tier return UNSUPPORTED. */
 #define NVFP4_PLAN_ACT_NVFP4  0x2000u
 #define NVFP4_PLAN_EPI_MASK   0xF00u
 #define NVFP4_PLAN_EPI_SWIGLU 0x100u

@@ -114,6 +114,7 @@ struct Params {
   int tpc;                                   // whole tiles per CTA (no split tiles), 0: stream-K
   int act4;                                  // W4A4: X quantised to NVFP4 in the kernel
   const float* row_scale;                    // FP8 tier: fp32 scale of each weight row [N]
+  const float* xgs;                          // W4A4 with X in the ring: gs_x written by k_xprep
   int xbytes, xbox_words, xbox_bytes;        // X in the ring: stage area, words per column, box bytes
   const int* xemax;                          // X in the ring: per-token exponent maximum
   const uint32_t* xlo;                       // X in the ring: per-token "lo plane used"
@@ -379,7 +380,7 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
 // ring stage.
 __global__ void __launch_bounds__(256)
 k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ planes, int pitch,
-        int* __restrict__ emax_out, uint32_t* __restrict__ lo_out) {
+        int* __restrict__ emax_out, uint32_t* __restrict__ lo_out, int act4, float* __restrict__ gsx_out) {
   // The main kernel may launch now (it waits for this grid before it reads
   // the planes, and meanwhile streams weights); X may be the previous grid's
   // output.
@@ -389,6 +390,51 @@ k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ plan
   const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint4* row = reinterpret_cast<const uint4*>(x + size_t(m) * K);
   const int chunks = K / 8;
+  if (act4) {
+    // W4A4: the token's row quantised to NVFP4 by the weights' quantiser steps
+    // under gs_x = amax(|X|) / 2688 over all of X (every CTA takes it over all
+    // tokens, so all agree); the hi plane holds the exact f16 products
+    // e2m1 * e4m3, the lo plane zeros, the per-token factor is 1.
+    const uint4* all = reinterpret_cast<const uint4*>(x);
+    uint32_t mg = 0u;
+    for (int u = threadIdx.x; u < M * chunks; u += 256) mg = max(mg, bf16_mag_max8(all[u]));
+    mg = __reduce_max_sync(0xffffffffu, mg);
+    if (lane == 0) s_max[warp] = int(mg);
+    __syncthreads();
+    uint32_t amax_bits = 0u;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) amax_bits = max(amax_bits, uint32_t(s_max[w]));
+    const float gsx = __fdiv_rn(__uint_as_float(amax_bits << 16), 2688.0f);   // 6 * 448
+    uint8_t* ch = planes + size_t(m) * pitch;
+    uint8_t* cl = planes + size_t(M + m) * pitch;
+    for (int b = threadIdx.x; b < K / 16; b += 256) {
+      const uint4 xa = row[2 * b], xb = row[2 * b + 1];
+      const uint32_t wv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(wv[i] << 16);
+        v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+      }
+      uint32_t s_code, q[2];
+      quantize_block16(v, gsx, s_code, q);
+      const uint32_t sc = bcast_lo(e4m3x2_to_f16x2(s_code));
+      uint32_t h[8];
+      e2m1x8_to_f16x2x4(q[0], h);
+      e2m1x8_to_f16x2x4(q[1], h + 4);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        *reinterpret_cast<uint2*>(ch + x_off(16 * b + 4 * c)) = make_uint2(hmul2(h[2 * c], sc), hmul2(h[2 * c + 1], sc));
+        *reinterpret_cast<uint2*>(cl + x_off(16 * b + 4 * c)) = make_uint2(0u, 0u);
+      }
+    }
+    if (threadIdx.x == 0) {
+      emax_out[m] = 14;
+      lo_out[m] = 0u;
+      if (m == 0) *gsx_out = gsx;
+    }
+    return;
+  }
   uint32_t mag = 0u;
   for (int kc = threadIdx.x; kc < chunks; kc += 256) mag = max(mag, bf16_mag_max8(row[kc]));
   int mx = bf16_mag_exp(__reduce_max_sync(0xffffffffu, mag));
@@ -737,9 +783,10 @@ __device__ __forceinline__ void consume(const Params& p, uint8_t* sW, uint8_t* s
       }
     }
     if (p.act4) {
-      // W4A4: the per-tensor scale of the quantised X (staged X: emax sits in
-      // the CTA's misc area next to it)
-      const float gsx = *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(emax) - MISC_EMAX + MISC_XGS);
+      // W4A4: the per-tensor scale of the quantised X (X in the ring: from
+      // k_xprep in the workspace; staged X: in the CTA's misc area, next to emax)
+      const float gsx = XR ? *p.xgs
+                           : *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(emax) - MISC_EMAX + MISC_XGS);
 #pragma unroll
       for (int e = 0; e < 4; ++e) { v[e][0] *= gsx; v[e][1] *= gsx; }
     }
@@ -1284,7 +1331,6 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   // From XR_MIN_M: 2M columns would force several K-slices; X goes through
   // the ring.
   c.xr = c.M >= XR_MIN_M;
-  if (c.act4 && c.xr) return cudaErrorInvalidConfiguration;   // W4A4: staged X only
   // FP8 weights: staged X, no epilogue, no W4A4 (a 64 KB stage leaves no room for X boxes)
   if (c.fmt == FMT_FP8 && (c.xr || c.epi != EPI_NONE || c.act4)) return cudaErrorInvalidConfiguration;
   const int stage_bytes = w_bytes_of(c.fmt) + s_bytes_of(c.fmt);
@@ -1361,7 +1407,7 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   if (c.xr) {
     c.ws_x_off = ((partials_end + 255) / 256) * 256;
     c.ws_xmeta_off = c.ws_x_off + ((size_t(c.ncols) * c.x_pitch + 255) / 256) * 256;
-    c.ws_bytes = c.ws_xmeta_off + 128;
+    c.ws_bytes = c.ws_xmeta_off + 144;        // exponents [16], lo flags [16], W4A4 gs_x
   } else {
     c.ws_x_off = c.ws_xmeta_off = 0;
     c.ws_bytes = partials_end;
@@ -1402,6 +1448,7 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
   p.partials = c.split ? reinterpret_cast<float*>(wsb + c.ws_partials_off) : nullptr;
   p.xemax = c.xr ? reinterpret_cast<const int*>(wsb + c.ws_xmeta_off) : nullptr;
   p.xlo = c.xr ? reinterpret_cast<const uint32_t*>(wsb + c.ws_xmeta_off + 64) : nullptr;
+  p.xgs = c.xr ? reinterpret_cast<const float*>(wsb + c.ws_xmeta_off + 128) : nullptr;
   p.keys = reinterpret_cast<unsigned long long*>(wsb + c.ws_epi_off);
   p.done = reinterpret_cast<uint32_t*>(wsb + c.ws_epi_off + 128);
   p.timeout = timeout_cycles;
@@ -1421,7 +1468,8 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
     pc.numAttrs = pdl ? 1 : 0;
     cudaError_t e = cudaLaunchKernelEx(&pc, k_xprep, x, c.M, c.K, wsb + c.ws_x_off, c.x_pitch,
                                        reinterpret_cast<int*>(wsb + c.ws_xmeta_off),
-                                       reinterpret_cast<uint32_t*>(wsb + c.ws_xmeta_off + 64));
+                                       reinterpret_cast<uint32_t*>(wsb + c.ws_xmeta_off + 64), c.act4,
+                                       reinterpret_cast<float*>(wsb + c.ws_xmeta_off + 128));
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};

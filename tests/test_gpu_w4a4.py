@@ -19,6 +19,7 @@ pytestmark = pytest.mark.gpu
 
 
 def run_w4a4(w, X, flags=0):
+    """Y bits [M][N] of the W4A4 linear through the C ABI (MMA variant)."""
     M, K = X.shape
     plan = nv.nvfp4_linear_plan(M, w.N, K, torch.cuda.current_device(), nv.NVFP4_PLAN_ACT_NVFP4 | flags)
     try:
@@ -48,7 +49,9 @@ def weights(N, K, seed):
 @pytest.mark.parametrize("M,N,K", [(1, 520, 512), (2, 1000, 768), (3, 777, 1280), (4, 4097, 512),
                                    (1, 130 * 256 - 77, 512), (1, 34816, 5120), (2, 34816, 5120),
                                    (1, 5120, 17408),
-                                   (4, 1024, 17408)])     # X in K-slices: each CTA quantises its slice
+                                   (4, 1024, 17408),      # X in K-slices: each CTA quantises its slice
+                                   # M >= 5: X in the ring, quantised by the X-conversion kernel
+                                   (5, 129, 256), (8, 2339, 1280), (16, 34816, 5120), (16, 5120, 17408)])
 def test_w4a4_linear(M, N, K):
     w = weights(N, K, seed=N + K)
     X = synth.x_bf16_custom(synth.X_OUTLIERS, M, K, seed=K + M, n_outliers=8, gain=20.0)
@@ -72,8 +75,9 @@ def test_w4a4_differs_from_the_bf16_linear_as_the_oracle_does():
     assert err16 > 10 * err4
 
 
-def test_w4a4_doubling_x_doubles_y_exactly():
-    M, N, K = 2, 777, 1024
+@pytest.mark.parametrize("M", [2, 12])
+def test_w4a4_doubling_x_doubles_y_exactly(M):
+    N, K = 777, 1024
     w = weights(N, K, seed=6)
     X = synth.x_bf16_custom(synth.X_NORMAL, M, K, seed=7)
     X2 = oracle.bf16_round_array(2.0 * oracle.bf16_bits_to_f64(X))
@@ -93,7 +97,7 @@ def test_w4a4_zero_x_gives_zero_y_and_repeats():
 
 def test_w4a4_plan_limits():
     d = torch.cuda.current_device()
-    bad = [(5, 1024, 512, 0), (1, 1024, 512, nv.NVFP4_VARIANT_TC), (1, 1024, 512, nv.NVFP4_VARIANT_GEMV),
+    bad = [(1, 1024, 512, nv.NVFP4_VARIANT_TC), (1, 1024, 512, nv.NVFP4_VARIANT_GEMV),
            (1, 1024, 512, nv.NVFP4_VARIANT_ROW), (1, 1024, 512, nv.NVFP4_PLAN_WEIGHT_FP8)]
     for M, N, K, flags in bad:
         with pytest.raises(nv.Nvfp4Error) as e:
