@@ -439,7 +439,7 @@ def run_ours(args):
                  [("lm_head", m, "nvfp4", "none") for m in (1, 8, 16)] + \
                  [("verify", m, "nvfp4", "swiglu") for m in (1, 16)] + \
                  [("lm_head", m, "nvfp4", "argmax") for m in (1, 16)] + \
-                 [("verify", m, "fp8", "none") for m in (1, 2)] + \
+                 [("verify", m, "fp8", "none") for m in (1, 2, 16)] + \
                  [("down", 1, "fp8", "none"), ("lm_head", 1, "fp8", "none")] + \
                  [("verify", m, "w4a4", "none") for m in (1, 4)] + [("down", 1, "w4a4", "none")]
         base_us = {}

@@ -109,7 +109,7 @@ typedef struct nvfp4_plan_s* nvfp4_plan_t;
  *     largest fp32 value gs * acc[n] (not rounded to bf16), equal values
  *     going to the lower n. The plan's workspace holds the running maxima;
  *     it is left cleared after the run, like the counters. */
-/* FP8 weight tier (plan flag; variant MMA, M <= 4 and no epilogue, or ROW if
+/* FP8 weight tier (plan flag; variant MMA without an epilogue, or ROW if
  * forced or if MMA cannot take the shape, M <= 2): W is stored as E4M3
  * codes, one byte per element, with one fp32 scale per row, for comparison
  * with NVFP4 at the same shapes (page "Qwen3.8-27B-NVFP4-RTX5090 API &

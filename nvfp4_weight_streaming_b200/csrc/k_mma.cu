@@ -1291,6 +1291,10 @@ cudaError_t set_smem_attrs(int optin) {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(k_mma<3, true, EPI, FMT_NVFP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   if (e == cudaSuccess && EPI == EPI_NONE)
     e = cudaFuncSetAttribute(k_mma<1, false, EPI_NONE, FMT_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess && EPI == EPI_NONE)
+    e = cudaFuncSetAttribute(k_mma<2, true, EPI_NONE, FMT_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess && EPI == EPI_NONE)
+    e = cudaFuncSetAttribute(k_mma<3, true, EPI_NONE, FMT_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
   return e;
 }
 
@@ -1299,7 +1303,12 @@ template <int EPI>
 cudaError_t launch_main(const MmaConfig& c, cudaLaunchConfig_t* cfg, const CUtensorMap& mw, const CUtensorMap& ms,
                         const CUtensorMap& mx, const mm::Params& p) {
   using namespace mm;
-  if (c.fmt == FMT_FP8) return cudaLaunchKernelEx(cfg, k_mma<1, false, EPI_NONE, FMT_FP8>, mw, ms, mx, p);
+  if (c.fmt == FMT_FP8) {
+    if (c.M <= 4 && !c.xr) return cudaLaunchKernelEx(cfg, k_mma<1, false, EPI_NONE, FMT_FP8>, mw, ms, mx, p);
+    if (c.M >= XR_MIN_M && c.M <= 8) return cudaLaunchKernelEx(cfg, k_mma<2, true, EPI_NONE, FMT_FP8>, mw, ms, mx, p);
+    if (c.M > 8) return cudaLaunchKernelEx(cfg, k_mma<3, true, EPI_NONE, FMT_FP8>, mw, ms, mx, p);
+    return cudaErrorInvalidConfiguration;
+  }
   if (c.M <= 4) {
     if (c.xr) return cudaLaunchKernelEx(cfg, k_mma<1, true, EPI, FMT_NVFP4>, mw, ms, mx, p);
     return cudaLaunchKernelEx(cfg, k_mma<1, false, EPI, FMT_NVFP4>, mw, ms, mx, p);
@@ -1331,9 +1340,11 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   // From XR_MIN_M: 2M columns would force several K-slices; X goes through
   // the ring.
   c.xr = c.M >= XR_MIN_M;
-  // FP8 weights: staged X, no epilogue, no W4A4 (a 64 KB stage leaves no room for X boxes)
-  if (c.fmt == FMT_FP8 && (c.xr || c.epi != EPI_NONE || c.act4)) return cudaErrorInvalidConfiguration;
+  // FP8 weights: no epilogue, no W4A4. With X in the ring a 64 KB stage and
+  // its X box leave room for two stages (still double-buffered).
+  if (c.fmt == FMT_FP8 && (c.epi != EPI_NONE || c.act4)) return cudaErrorInvalidConfiguration;
   const int stage_bytes = w_bytes_of(c.fmt) + s_bytes_of(c.fmt);
+  const int nstage_min = (c.fmt == FMT_FP8 && c.xr) ? 2 : NSTAGE_MIN;
   int S = 1;
   if (c.xr) {
     c.x_box = 4 * XGROUP_BYTES;
@@ -1392,7 +1403,7 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
     int nst = int(left / (stage_bytes + c.xbytes));
     c.nstage = nst < NSTAGE_MAX ? nst : NSTAGE_MAX;
   }
-  if (c.nstage < NSTAGE_MIN) return cudaErrorInvalidConfiguration;
+  if (c.nstage < nstage_min) return cudaErrorInvalidConfiguration;
   c.smem = 1024 + size_t(c.nstage) * (stage_bytes + c.xbytes) +
            (c.xr ? 0 : size_t(c.ncols) * c.xstride) + misc_bytes(c.M);
   if (c.smem > size_t(optin)) return cudaErrorInvalidConfiguration;

@@ -4,8 +4,8 @@ The tier stores W as E4M3 codes [N][K] with one fp32 scale per row (reading
 R15: s_n = amax|W[n]| / 448, code = E4M3_RNE_satfinite(w / s_n)); the GPU
 quantiser must reproduce the oracle's codes and scales bit for bit, and the
 linear must meet the stated tolerance against the oracle's fp64 sum of
-e4m3(code) * s_n * x. Runs on the MMA variant (the default, M <= 4) and on the
-row-block variant (forced, M <= 2).
+e4m3(code) * s_n * x. Runs on the MMA variant (the default, every M) and on
+the row-block variant (forced, M <= 2).
 """
 import numpy as np
 import pytest
@@ -84,7 +84,9 @@ def run_fp8(codes, sc, X, gs=1.0, repeat=1, variant=0):
 
 @pytest.mark.parametrize("M,N,K", [(1, 520, 512), (2, 1000, 768), (1, 2, 256), (2, 2339, 5120),
                                    (1, 34816, 5120), (1, 5120, 17408), (3, 777, 1280),
-                                   (4, 130 * 256 - 77, 512)])
+                                   (4, 130 * 256 - 77, 512),
+                                   # X in the ring (M >= 5)
+                                   (5, 129, 256), (8, 2339, 1280), (16, 34816, 5120), (16, 5120, 17408)])
 @pytest.mark.parametrize("variant", [0, nv.NVFP4_VARIANT_ROW])
 def test_fp8_linear(M, N, K, variant):
     if variant == nv.NVFP4_VARIANT_ROW and M > 2:
@@ -161,12 +163,13 @@ def test_fp8_plan_limits():
         with pytest.raises(nv.Nvfp4Error) as e:
             nv.nvfp4_linear_plan(1, 1024, 512, d, flags)
         assert e.value.status == nv.NVFP4_ERR_UNSUPPORTED
-    for M, flags in ((5, 0), (3, nv.NVFP4_VARIANT_ROW)):
+    for M, flags in ((5, nv.NVFP4_VARIANT_ROW), (3, nv.NVFP4_VARIANT_ROW)):
         with pytest.raises(nv.Nvfp4Error) as e:
             nv.nvfp4_linear_plan(M, 1024, 512, d, nv.NVFP4_PLAN_WEIGHT_FP8 | flags)
         assert e.value.status == nv.NVFP4_ERR_UNSUPPORTED
-    p = nv.nvfp4_linear_plan(4, 1024, 512, d, nv.NVFP4_PLAN_WEIGHT_FP8)
-    try:
-        assert nv.nvfp4_linear_variant(p) == nv.NVFP4_VARIANT_MMA
-    finally:
-        nv.nvfp4_linear_destroy(p)
+    for M in (4, 16):
+        p = nv.nvfp4_linear_plan(M, 1024, 512, d, nv.NVFP4_PLAN_WEIGHT_FP8)
+        try:
+            assert nv.nvfp4_linear_variant(p) == nv.NVFP4_VARIANT_MMA
+        finally:
+            nv.nvfp4_linear_destroy(p)
