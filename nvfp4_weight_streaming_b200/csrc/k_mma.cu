@@ -85,7 +85,6 @@ constexpr int NSTAGE_MIN = 3;             // ring depth the X budget is planned 
 constexpr int NSTAGE_MAX = 8;             // deeper rings use what X leaves free
 constexpr int W_BYTES = TROWS * KS / 2;    // 32768
 constexpr int S_BYTES = TROWS * KS / 16;   // 4096
-constexpr int STAGE_BYTES = W_BYTES + S_BYTES;
 // FP8 weight tier: E4M3 codes [N][K], one fp32 scale per row; a stage holds
 // 256 rows x 256 codes as two 128-byte-wide swizzled halves (K 0..127, 128..255)
 constexpr int FMT_NVFP4 = 0, FMT_FP8 = 1;
@@ -378,9 +377,17 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
 // layout of x_off) and records the token's exponent maximum and whether its
 // lo plane is used. The main kernel then loads one K-step of all planes per
 // ring stage.
-__global__ void __launch_bounds__(256)
+//
+// Both conversion kernels are held to 32 registers a thread: the main kernel
+// triggers its launch at the top of theirs, and with 18 warps of 82-88
+// registers it leaves 2304 registers in an SM sub-partition of 16384, two
+// warps of up to 32 each. Above that a conversion block cannot share an SM
+// with a main CTA; with a main grid on every SM each call then waits for SMs
+// to drain (measured: +9 us a call on the down projection at M = 8 and 16
+// with 43 registers, none at 32).
+__global__ void __launch_bounds__(256, 8)
 k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ planes, int pitch,
-        int* __restrict__ emax_out, uint32_t* __restrict__ lo_out, int act4, float* __restrict__ gsx_out) {
+        int* __restrict__ emax_out, uint32_t* __restrict__ lo_out) {
   // The main kernel may launch now (it waits for this grid before it reads
   // the planes, and meanwhile streams weights); X may be the previous grid's
   // output.
@@ -390,51 +397,6 @@ k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ plan
   const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint4* row = reinterpret_cast<const uint4*>(x + size_t(m) * K);
   const int chunks = K / 8;
-  if (act4) {
-    // W4A4: the token's row quantised to NVFP4 by the weights' quantiser steps
-    // under gs_x = amax(|X|) / 2688 over all of X (every CTA takes it over all
-    // tokens, so all agree); the hi plane holds the exact f16 products
-    // e2m1 * e4m3, the lo plane zeros, the per-token factor is 1.
-    const uint4* all = reinterpret_cast<const uint4*>(x);
-    uint32_t mg = 0u;
-    for (int u = threadIdx.x; u < M * chunks; u += 256) mg = max(mg, bf16_mag_max8(all[u]));
-    mg = __reduce_max_sync(0xffffffffu, mg);
-    if (lane == 0) s_max[warp] = int(mg);
-    __syncthreads();
-    uint32_t amax_bits = 0u;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) amax_bits = max(amax_bits, uint32_t(s_max[w]));
-    const float gsx = __fdiv_rn(__uint_as_float(amax_bits << 16), 2688.0f);   // 6 * 448
-    uint8_t* ch = planes + size_t(m) * pitch;
-    uint8_t* cl = planes + size_t(M + m) * pitch;
-    for (int b = threadIdx.x; b < K / 16; b += 256) {
-      const uint4 xa = row[2 * b], xb = row[2 * b + 1];
-      const uint32_t wv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-      float v[16];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        v[2 * i] = __uint_as_float(wv[i] << 16);
-        v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
-      }
-      uint32_t s_code, q[2];
-      quantize_block16(v, gsx, s_code, q);
-      const uint32_t sc = bcast_lo(e4m3x2_to_f16x2(s_code));
-      uint32_t h[8];
-      e2m1x8_to_f16x2x4(q[0], h);
-      e2m1x8_to_f16x2x4(q[1], h + 4);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        *reinterpret_cast<uint2*>(ch + x_off(16 * b + 4 * c)) = make_uint2(hmul2(h[2 * c], sc), hmul2(h[2 * c + 1], sc));
-        *reinterpret_cast<uint2*>(cl + x_off(16 * b + 4 * c)) = make_uint2(0u, 0u);
-      }
-    }
-    if (threadIdx.x == 0) {
-      emax_out[m] = 14;
-      lo_out[m] = 0u;
-      if (m == 0) *gsx_out = gsx;
-    }
-    return;
-  }
   uint32_t mag = 0u;
   for (int kc = threadIdx.x; kc < chunks; kc += 256) mag = max(mag, bf16_mag_max8(row[kc]));
   int mx = bf16_mag_exp(__reduce_max_sync(0xffffffffu, mag));
@@ -461,6 +423,59 @@ k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ plan
   if (threadIdx.x == 0) {
     emax_out[m] = emax;
     lo_out[m] = lo_used ? 1u : 0u;
+  }
+}
+
+// W4A4 with X in the ring: the token's row quantised to NVFP4 by the weights'
+// quantiser steps under gs_x = amax(|X|) / 2688 over all of X (every CTA takes
+// the maximum over all tokens, so all agree); the hi plane holds the exact f16
+// products e2m1 * e4m3, the lo plane zeros, the per-token factor is 1, and
+// CTA 0 stores gs_x for the main kernel's epilogue.
+__global__ void __launch_bounds__(256, 8)
+k_xprep_act4(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ planes, int pitch,
+             int* __restrict__ emax_out, uint32_t* __restrict__ lo_out, float* __restrict__ gsx_out) {
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  __shared__ uint32_t s_max[8];
+  const int m = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint4* row = reinterpret_cast<const uint4*>(x + size_t(m) * K);
+  const uint4* all = reinterpret_cast<const uint4*>(x);
+  uint32_t mg = 0u;
+  for (int u = threadIdx.x; u < M * (K / 8); u += 256) mg = max(mg, bf16_mag_max8(all[u]));
+  mg = __reduce_max_sync(0xffffffffu, mg);
+  if (lane == 0) s_max[warp] = mg;
+  __syncthreads();
+  uint32_t amax_bits = 0u;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) amax_bits = max(amax_bits, s_max[w]);
+  const float gsx = __fdiv_rn(__uint_as_float(amax_bits << 16), 2688.0f);   // 6 * 448
+  uint8_t* ch = planes + size_t(m) * pitch;
+  uint8_t* cl = planes + size_t(M + m) * pitch;
+  for (int b = threadIdx.x; b < K / 16; b += 256) {
+    const uint4 xa = row[2 * b], xb = row[2 * b + 1];
+    const uint32_t wv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      v[2 * i] = __uint_as_float(wv[i] << 16);
+      v[2 * i + 1] = __uint_as_float(wv[i] & 0xFFFF0000u);
+    }
+    uint32_t s_code, q[2];
+    quantize_block16(v, gsx, s_code, q);
+    const uint32_t sc = bcast_lo(e4m3x2_to_f16x2(s_code));
+    uint32_t h[8];
+    e2m1x8_to_f16x2x4(q[0], h);
+    e2m1x8_to_f16x2x4(q[1], h + 4);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      *reinterpret_cast<uint2*>(ch + x_off(16 * b + 4 * c)) = make_uint2(hmul2(h[2 * c], sc), hmul2(h[2 * c + 1], sc));
+      *reinterpret_cast<uint2*>(cl + x_off(16 * b + 4 * c)) = make_uint2(0u, 0u);
+    }
+  }
+  if (threadIdx.x == 0) {
+    emax_out[m] = 14;
+    lo_out[m] = 0u;
+    if (m == 0) *gsx_out = gsx;
   }
 }
 
@@ -1477,10 +1492,12 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
     pc.stream = st;
     pc.attrs = attr;
     pc.numAttrs = pdl ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&pc, k_xprep, x, c.M, c.K, wsb + c.ws_x_off, c.x_pitch,
-                                       reinterpret_cast<int*>(wsb + c.ws_xmeta_off),
-                                       reinterpret_cast<uint32_t*>(wsb + c.ws_xmeta_off + 64), c.act4,
-                                       reinterpret_cast<float*>(wsb + c.ws_xmeta_off + 128));
+    int* emax = reinterpret_cast<int*>(wsb + c.ws_xmeta_off);
+    uint32_t* lo = reinterpret_cast<uint32_t*>(wsb + c.ws_xmeta_off + 64);
+    cudaError_t e =
+        c.act4 ? cudaLaunchKernelEx(&pc, k_xprep_act4, x, c.M, c.K, wsb + c.ws_x_off, c.x_pitch, emax, lo,
+                                    reinterpret_cast<float*>(wsb + c.ws_xmeta_off + 128))
+               : cudaLaunchKernelEx(&pc, k_xprep, x, c.M, c.K, wsb + c.ws_x_off, c.x_pitch, emax, lo);
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
