@@ -440,11 +440,17 @@ def run_ours(args):
                  [("verify", m, "nvfp4", "swiglu") for m in (1, 16)] + \
                  [("lm_head", m, "nvfp4", "argmax") for m in (1, 16)] + \
                  [("verify", m, "fp8", "none") for m in (1, 2, 16)] + \
-                 [("down", 1, "fp8", "none"), ("lm_head", 1, "fp8", "none")] + \
-                 [("verify", m, "w4a4", "none") for m in (1, 4)] + [("down", 1, "w4a4", "none")]
+                 [("down", 1, "fp8", "none"), ("lm_head", 1, "fp8", "none")]
+        points = [pt + (None,) for pt in points]
+        # W4A4 on both of its variants: decoded for the warp MMA, and the
+        # block-scaled FP4 tensor cores
+        for v4 in (nv.NVFP4_VARIANT_MMA, nv.NVFP4_VARIANT_TC):
+            points += [("verify", m, "w4a4", "none", v4) for m in (1, 4, 16)] + \
+                      [("down", m, "w4a4", "none", v4) for m in (1, 16)]
+        points += [("lm_head", 1, "w4a4", "none", nv.NVFP4_VARIANT_TC)]
         base_us = {}
-        for (name, M, fmt, epi) in points:
-            v = variant if (fmt == "nvfp4" and epi == "none") else 0
+        for (name, M, fmt, epi, forced) in points:
+            v = forced if forced is not None else variant if (fmt == "nvfp4" and epi == "none") else 0
             q = Problem(name, M, v, min_footprint=4.2 * l2, flags=flags, fmt=fmt, epi=epi)
             s2, _, r2 = time_problem(q, max(args.steps, 200), args.warmup, world, repeats=args.repeats)
             g = effective_gbs(q.bytes, s2)

@@ -121,23 +121,32 @@ typedef struct nvfp4_plan_s* nvfp4_plan_t;
  * the tolerance and the X range are as for NVFP4. nvfp4_quantize_fp8 makes
  * such weights. */
 #define NVFP4_PLAN_WEIGHT_FP8 0x1000u
-/* W4A4 tier (plan flag; MMA variant, any M): X arrives as bf16 like
- * always and is quantised to NVFP4 inside the kernel with the weights'
+/* W4A4 tier (plan flag; variants MMA and TC, any M): X arrives as bf16 like
+ * always and is quantised to NVFP4 on the device with the weights'
  * quantiser steps -- 16-element blocks of a token row, E4M3 block scales,
  * one per-tensor scale gs_x = amax(|X|) / (6 * 448) of the call's X (page
  * "Qwen3.8-27B-NVFP4-RTX5090 API & Inference Endpoint", section "Recipe
  * (NVIDIA ModelOpt)": weights and activations NVFP4). Y is then sum_k
  * w_hat[n][k] * x_hat[m][k] with x_hat = e2m1 * e4m3 * gs_x: a different
  * (quantised) result from the W4A16 linear; the same tolerance, against the
- * fp64 sum of w_hat * x_hat, applies. For M <= 4 every CTA quantises the
- * K-steps it stages; from M = 5 the X-conversion kernel quantises X once per
- * call. Other variants and the FP8 weight tier return UNSUPPORTED. */
+ * fp64 sum of w_hat * x_hat, applies.
+ *   MMA: codes decoded to f16 for the warp MMA; for M <= 4 every CTA
+ *     quantises the K-steps it stages, from M = 5 the X-conversion kernel
+ *     quantises X once per call. Takes the fused epilogues.
+ *   TC: the block-scaled FP4 tensor cores (tcgen05.mma kind::mxf4nvf4) read
+ *     the packed codes as stored and apply the block scales themselves; two
+ *     small kernels quantise X first (3 launches per call). The scale bytes
+ *     are read as unsigned E4M3: their sign bit must be clear (nvfp4_quantize
+ *     never sets it). No fused epilogue.
+ * AUTO takes TC from M = 4 without an epilogue (its time is flat in M) and
+ * MMA otherwise, or MMA when TC cannot take the plan. GEMV, ROW and the FP8
+ * weight tier return UNSUPPORTED. */
 #define NVFP4_PLAN_ACT_NVFP4  0x2000u
 #define NVFP4_PLAN_EPI_MASK   0xF00u
 #define NVFP4_PLAN_EPI_SWIGLU 0x100u
 #define NVFP4_PLAN_EPI_ARGMAX 0x200u
-/* Programmatic dependent launch (MMA and ROW variants; ignored by the
- * others). The launch may start while the previous kernel in the stream is
+/* Programmatic dependent launch (MMA and ROW variants and W4A4 on TC;
+ * ignored by the others). The launch may start while the previous kernel in the stream is
  * still running:
  * it begins streaming W at once and touches X, Y, w_global and the workspace
  * only after that kernel has completed. So W (codes and scales) must not be
@@ -183,8 +192,9 @@ int nvfp4_auto_variant(int M, int N, int K);
 /* Kernels one nvfp4_linear_run (or nvfp4_linear_run_static) of this plan
  * launches: 2 for the mma variant when X goes through its ring (M >= 5, or a
  * K so long that X does not fit next to the ring: X is converted to its two
- * f16 planes by a kernel of its own first), 1 otherwise, 0 when N == 0; -1
- * if the plan is null. Host-only; touches no device. */
+ * f16 planes by a kernel of its own first), 3 for a W4A4 plan on the TC
+ * variant (X amax, X quantisation, the linear), 1 otherwise, 0 when N == 0;
+ * -1 if the plan is null. Host-only; touches no device. */
 int nvfp4_linear_launches_per_run(nvfp4_plan_t plan);
 
 /* Run the linear on `stream` (device pointers, see the layout above):

@@ -40,6 +40,7 @@ struct nvfp4_plan_s {
   size_t ws_bytes;
   nvfp4::GemvConfig gemv;
   nvfp4::TcConfig tc;
+  nvfp4::Tc4Config tc4;   // TC variant of a W4A4 plan
   nvfp4::MmaConfig mma;
   nvfp4::RowConfig row;
   std::mutex map_mu;
@@ -123,7 +124,10 @@ bool lookup_maps(nvfp4_plan_s* p, const void* wp, const void* ws, CUtensorMap* m
     ok = nvfp4::encode_fp8_codes_map(p->N, p->K, static_cast<const uint8_t*>(wp), &e.mw);
     e.ms = e.mw;
   } else {
-    const int box_rows = p->variant == int(NVFP4_VARIANT_MMA) ? nvfp4::kMmaTileRows : 128;
+    // 256-row boxes for the MMA variant and the W4A4 tensor-core kernel, 128 for TC
+    const int box_rows =
+        (p->variant == int(NVFP4_VARIANT_MMA) || (p->variant == int(NVFP4_VARIANT_TC) && p->act4))
+            ? nvfp4::kMmaTileRows : 128;
     ok = nvfp4::encode_weight_maps(p->N, p->K, box_rows, static_cast<const uint8_t*>(wp),
                                    static_cast<const uint8_t*>(ws), &e.mw, &e.ms);
   }
@@ -194,8 +198,12 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   p.split_k = 1;
   p.ws_bytes = 0;
   unsigned forced = flags & NVFP4_PLAN_VARIANT_MASK;
+  // W4A4: the block-scaled FP4 tensor cores from M = 4 on (their time is flat
+  // in M), the warp-MMA kernel below that and for the fused epilogues
   p.variant = forced ? int(forced)
-                     : (fmt == 1 || act4 ? int(NVFP4_VARIANT_MMA) : auto_variant(M, N, K));
+              : fmt == 1 ? int(NVFP4_VARIANT_MMA)
+              : act4     ? ((M >= 4 && epi == 0) ? int(NVFP4_VARIANT_TC) : int(NVFP4_VARIANT_MMA))
+                         : auto_variant(M, N, K);
   if (K == 0 || N == 0) {
     // nothing to contract: run() writes zeros (K == 0) or returns (N == 0)
     if (p.variant == int(NVFP4_VARIANT_GEMV) && M > 4) p.variant = int(NVFP4_VARIANT_TC);
@@ -206,7 +214,8 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
     if (p.fmt != 0 && ((p.variant != int(NVFP4_VARIANT_ROW) && p.variant != int(NVFP4_VARIANT_MMA)) ||
                        p.epi != 0 || p.act4 != 0))
       return NVFP4_ERR_UNSUPPORTED;
-    if (p.act4 && p.variant != int(NVFP4_VARIANT_MMA)) return NVFP4_ERR_UNSUPPORTED;
+    if (p.act4 && p.variant != int(NVFP4_VARIANT_MMA) && p.variant != int(NVFP4_VARIANT_TC))
+      return NVFP4_ERR_UNSUPPORTED;
     switch (p.variant) {
       case NVFP4_VARIANT_GEMV: {
         if (M > 4 || size_t(M) * size_t(K) * 4 > 200 * 1024) { st = NVFP4_ERR_UNSUPPORTED; break; }
@@ -238,6 +247,15 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
       }
       case NVFP4_VARIANT_TC: {
         if (K == 0 || N == 0) break;
+        if (p.act4) {
+          p.tc4.M = M; p.tc4.N = N; p.tc4.K = K;
+          cudaError_t e = nvfp4::tc4_configure(p.tc4, sms);
+          if (e == cudaErrorNotSupported || e == cudaErrorInvalidConfiguration) st = NVFP4_ERR_UNSUPPORTED;
+          else if (e != cudaSuccess) st = NVFP4_ERR_CUDA;
+          p.split_k = p.tc4.S;
+          p.ws_bytes = p.tc4.ws_bytes;
+          break;
+        }
         p.tc.M = M; p.tc.N = N; p.tc.K = K;
         cudaError_t e = nvfp4::tc_configure(p.tc, sms);
         if (e == cudaErrorNotSupported || e == cudaErrorInvalidConfiguration) st = NVFP4_ERR_UNSUPPORTED;
@@ -255,6 +273,12 @@ nvfp4_status nvfp4_linear_plan(int M, int N, int K, int device, unsigned flags,
   if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.fmt == 1 && p.variant == int(NVFP4_VARIANT_MMA)) {
     // FP8 weights the MMA variant cannot take (X does not fit beside its ring): the row variant
     p.variant = int(NVFP4_VARIANT_ROW);
+    p.split_k = 1;
+    p.ws_bytes = 0;
+    st = configure();
+  }
+  if (st == NVFP4_ERR_UNSUPPORTED && !forced && p.act4 && p.variant == int(NVFP4_VARIANT_TC)) {
+    p.variant = int(NVFP4_VARIANT_MMA);
     p.split_k = 1;
     p.ws_bytes = 0;
     st = configure();
@@ -293,6 +317,7 @@ int nvfp4_linear_launches_per_run(nvfp4_plan_t plan) {
   if (!plan) return -1;
   if (plan->N == 0) return 0;
   if (plan->K > 0 && plan->variant == NVFP4_VARIANT_MMA && plan->mma.xr) return 2;
+  if (plan->K > 0 && plan->variant == NVFP4_VARIANT_TC && plan->act4) return 3;
   return 1;
 }
 
@@ -367,6 +392,12 @@ nvfp4_status nvfp4_linear_run(nvfp4_plan_t plan, const uint8_t* w_packed,
         CUtensorMap mw, ms;
         if (!lookup_maps(plan, w_packed, w_scales, &mw, &ms)) return NVFP4_ERR_CUDA;
         const bool stall = (plan->flags & NVFP4_PLAN_TEST_STALL) != 0;
+        if (plan->act4) {
+          const bool pdl = (plan->flags & NVFP4_PLAN_PDL) != 0;
+          e = nvfp4::launch_tc4(plan->tc4, &mw, &ms, w_global, xb, yb, workspace,
+                                stall ? kStallTimeoutCycles : kTimeoutCycles, stall, pdl, st);
+          break;
+        }
         e = nvfp4::launch_tc(plan->tc, &mw, &ms, w_global, xb, yb, workspace,
                              stall ? kStallTimeoutCycles : kTimeoutCycles, stall, st);
         break;

@@ -56,6 +56,20 @@ cudaError_t launch_tc(const TcConfig& c, const void* map_w, const void* map_s, c
                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles,
                       bool stall, cudaStream_t st);
 
+// W4A4 on the block-scaled FP4 tensor cores (k_tc4.cu): X quantised to NVFP4
+// once per call into the workspace, tcgen05.mma kind::mxf4nvf4 on the raw
+// codes with the E4M3 block scales in tensor memory. Three launches per call.
+struct Tc4Config {
+  int M, N, K;
+  int tiles, S, ks_base, ks_rem, units, grid;
+  size_t smem, ws_amax_off, ws_gsx_off, ws_counters_off, ws_x_off, ws_partials_off, ws_bytes;
+};
+cudaError_t tc4_configure(Tc4Config& c, int num_sms);
+// map_w / map_s: encode_weight_maps with 256-row boxes.
+cudaError_t launch_tc4(const Tc4Config& c, const void* map_w, const void* map_s, const float* gs,
+                       const uint16_t* x, uint16_t* y, void* workspace, long long timeout_cycles, bool stall,
+                       bool pdl, cudaStream_t st);
+
 // Register-direct warp-MMA variant (k_mma.cu).
 struct MmaConfig {
   int M, N, K;
