@@ -387,7 +387,7 @@ def measured_traffic(variant: str, workload: str):
     record (profiles/traffic.json), or None when the kernel's sources have
     changed since the capture or the capture was of another workload."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    kernel = {"mma": "k_mma"}.get(variant)
+    kernel = {"mma": "k_mma", "w4a4-tc": "k_tc4"}.get(variant)
     if kernel is None or not os.path.exists(path):
         return None
     rec = json.load(open(path)).get(kernel)
@@ -421,7 +421,7 @@ def run_ours(args):
     peak, peak_kind = peaks()
     variant = {"auto": 0, "gemv": 1, "mma": 2, "tc": 3, "row": 4}[args.variant]
     flags = 0 if args.no_pdl else nv.NVFP4_PLAN_PDL
-    pb = Problem(args.workload, args.M, variant, min_footprint=4.2 * l2, flags=flags)
+    pb = Problem(args.workload, args.M, variant, min_footprint=4.2 * l2, flags=flags, fmt=args.fmt)
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if sampler:
         sampler.start()
@@ -484,10 +484,13 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
             "repeats": len(reps), "ms_per_step_spread": [min(reps) * 1e3, max(reps) * 1e3],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "nvfp4 weights x bf16 activations, f16 products, f32 accumulate",
+            "dtype": {"nvfp4": "nvfp4 weights x bf16 activations, f16 products, f32 accumulate",
+                      "w4a4": "nvfp4 weights x nvfp4 activations (quantised on the device), "
+                              "f32 accumulate",
+                      "fp8": "e4m3 weights x bf16 activations, f16 products, f32 accumulate"}[args.fmt],
             "data": "synthetic (seeded SplitMix64/Box-Muller, workload recipes in synth/)",
             "config": {"workload": "%s projection M=%d K=%d N=%d" % (args.workload, pb.M, pb.K, pb.N),
-                       "M": pb.M, "K": pb.K, "N": pb.N,
+                       "M": pb.M, "K": pb.K, "N": pb.N, "tier": args.fmt,
                        "variant": VARIANT_NAMES[pb.variant],
                        "split_k": pb.split_k, "bytes_per_call": pb.bytes,
                        "l2": "inputs larger than L2: %d byte-identical weight copies "
@@ -502,7 +505,8 @@ def run_ours(args):
             "pct_of_nominal_8TBps": 100 * per_gpu / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peak, "unit": "GB/s",
                          "frac": per_gpu / peak,
-                         "traffic": measured_traffic(VARIANT_NAMES[pb.variant],
+                         "traffic": measured_traffic(VARIANT_NAMES[pb.variant] if args.fmt == "nvfp4"
+                                                     else args.fmt + "-" + VARIANT_NAMES[pb.variant],
                                                      "%s projection M=%d K=%d N=%d" %
                                                      (args.workload, pb.M, pb.K, pb.N)),
                          "peak_kind": peak_kind + " device-copy bandwidth (MEASURED_PEAKS hbm_gbs)"},
@@ -593,6 +597,9 @@ def main():
     ap.add_argument("--workload", default="decode")
     ap.add_argument("--M", type=int, default=1)
     ap.add_argument("--variant", choices=list(VARIANT_NAMES), default="auto")
+    ap.add_argument("--fmt", choices=["nvfp4", "w4a4", "fp8"], default="nvfp4",
+                    help="main problem's tier: NVFP4 weights with bf16 X (the method), X also "
+                         "quantised to NVFP4, or FP8 weights")
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-pdl", action="store_true",
                     help="launch without programmatic dependent launch")

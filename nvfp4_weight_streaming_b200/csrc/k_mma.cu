@@ -66,6 +66,7 @@
 #include "nvfp4_device.cuh"
 
 #include <cuda.h>
+#include <algorithm>
 #include <climits>
 #include <vector>
 
@@ -73,6 +74,7 @@ namespace nvfp4 {
 namespace mm {
 
 constexpr int KS = 256;                    // K elements per step
+constexpr int XP_STEPS = 8;                // K-steps one X-conversion block converts
 constexpr int TROWS = 256;                 // weight rows per tile
 constexpr int NCW = 16;                    // consumer warps (16 rows each)
 constexpr int WARP_SETTLE = NCW + 1;       // warp 0 producer, 1..16 consumers, 17 settler
@@ -116,7 +118,8 @@ struct Params {
   const float* xgs;                          // W4A4 with X in the ring: gs_x written by k_xprep
   int xbytes, xbox_words, xbox_bytes;        // X in the ring: stage area, words per column, box bytes
   const int* xemax;                          // X in the ring: per-token exponent maximum
-  const uint32_t* xlo;                       // X in the ring: per-token "lo plane used"
+  const uint32_t* xlo;                       // X in the ring: "lo plane used" [xchunks][16]
+  int xchunks;                               // X in the ring: conversion blocks per token
   const float* gs;
   const uint16_t* x;
   uint16_t* y;
@@ -385,9 +388,14 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
 // with a main CTA; with a main grid on every SM each call then waits for SMs
 // to drain (measured: +9 us a call on the down projection at M = 8 and 16
 // with 43 registers, none at 32).
+//
+// Block (m, c) of the grid (M, C) takes the maximum over the whole row but
+// converts only K-steps [csteps c, csteps (c + 1)), so a long row is
+// converted by several SMs at once; it records its lo-plane use in its own
+// slot lo_out[16 c + m] (the main kernel ORs the slots of a token).
 __global__ void __launch_bounds__(256, 8)
 k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ planes, int pitch,
-        int* __restrict__ emax_out, uint32_t* __restrict__ lo_out) {
+        int* __restrict__ emax_out, uint32_t* __restrict__ lo_out, int csteps) {
   // The main kernel may launch now (it waits for this grid before it reads
   // the planes, and meanwhile streams weights); X may be the previous grid's
   // output.
@@ -409,7 +417,8 @@ k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ plan
   bool lo_used = false;
   uint8_t* ch = planes + size_t(m) * pitch;
   uint8_t* cl = planes + size_t(M + m) * pitch;
-  for (int kc = threadIdx.x; kc < chunks; kc += 256) {
+  const int kc_end = min(chunks, int(blockIdx.y + 1) * (csteps * KS / 8));
+  for (int kc = int(blockIdx.y) * (csteps * KS / 8) + threadIdx.x; kc < kc_end; kc += 256) {
     const uint4 v = row[kc];
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t hi[4], lo[4];
@@ -421,8 +430,8 @@ k_xprep(const uint16_t* __restrict__ x, int M, int K, uint8_t* __restrict__ plan
   }
   lo_used = __syncthreads_or(lo_used);
   if (threadIdx.x == 0) {
-    emax_out[m] = emax;
-    lo_out[m] = lo_used ? 1u : 0u;
+    emax_out[m] = emax;                        // the same value from every block of the row
+    lo_out[16 * blockIdx.y + m] = lo_used ? 1u : 0u;
   }
 }
 
@@ -1115,7 +1124,8 @@ k_mma(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
     if constexpr (XR) {
       // X arrives with the weights; exponents and lo flags come from k_xprep
       bool need_lo = false;
-      for (int m = 0; m < p.M; ++m) need_lo |= p.xlo[m] != 0u;
+      for (int c = 0; c < p.xchunks; ++c)
+        for (int m = 0; m < p.M; ++m) need_lo |= p.xlo[16 * c + m] != 0u;
       if constexpr (MC == 1) {
         if (FMT == FMT_NVFP4 && (p.M == 1 || (p.M == 2 && !need_lo))) NVFP4_CONSUME(0, 1, false, true, p.xemax);
         else if (need_lo) NVFP4_CONSUME(1, 1, true, true, p.xemax); else NVFP4_CONSUME(1, 1, false, true, p.xemax);
@@ -1433,7 +1443,9 @@ cudaError_t mma_configure(MmaConfig& c, int num_sms) {
   if (c.xr) {
     c.ws_x_off = ((partials_end + 255) / 256) * 256;
     c.ws_xmeta_off = c.ws_x_off + ((size_t(c.ncols) * c.x_pitch + 255) / 256) * 256;
-    c.ws_bytes = c.ws_xmeta_off + 144;        // exponents [16], lo flags [16], W4A4 gs_x
+    // exponents [16], W4A4 gs_x, lo flags [xchunks][16]
+    c.xchunks = c.act4 ? 1 : std::min(16, (c.K / KS + XP_STEPS - 1) / XP_STEPS);
+    c.ws_bytes = c.ws_xmeta_off + 128 + size_t(c.xchunks) * 64;
   } else {
     c.ws_x_off = c.ws_xmeta_off = 0;
     c.ws_bytes = partials_end;
@@ -1473,8 +1485,9 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
   p.counters = reinterpret_cast<uint32_t*>(wsb + c.ws_counters_off);
   p.partials = c.split ? reinterpret_cast<float*>(wsb + c.ws_partials_off) : nullptr;
   p.xemax = c.xr ? reinterpret_cast<const int*>(wsb + c.ws_xmeta_off) : nullptr;
-  p.xlo = c.xr ? reinterpret_cast<const uint32_t*>(wsb + c.ws_xmeta_off + 64) : nullptr;
-  p.xgs = c.xr ? reinterpret_cast<const float*>(wsb + c.ws_xmeta_off + 128) : nullptr;
+  p.xlo = c.xr ? reinterpret_cast<const uint32_t*>(wsb + c.ws_xmeta_off + 128) : nullptr;
+  p.xgs = c.xr ? reinterpret_cast<const float*>(wsb + c.ws_xmeta_off + 64) : nullptr;
+  p.xchunks = c.xr ? c.xchunks : 0;
   p.keys = reinterpret_cast<unsigned long long*>(wsb + c.ws_epi_off);
   p.done = reinterpret_cast<uint32_t*>(wsb + c.ws_epi_off + 128);
   p.timeout = timeout_cycles;
@@ -1487,17 +1500,18 @@ cudaError_t launch_mma(const MmaConfig& c, const void* map_w, const void* map_s,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   if (c.xr) {
     cudaLaunchConfig_t pc = {};
-    pc.gridDim = dim3(c.M);
+    pc.gridDim = dim3(c.M, c.xchunks);
     pc.blockDim = dim3(256);
     pc.stream = st;
     pc.attrs = attr;
     pc.numAttrs = pdl ? 1 : 0;
     int* emax = reinterpret_cast<int*>(wsb + c.ws_xmeta_off);
-    uint32_t* lo = reinterpret_cast<uint32_t*>(wsb + c.ws_xmeta_off + 64);
+    uint32_t* lo = reinterpret_cast<uint32_t*>(wsb + c.ws_xmeta_off + 128);
     cudaError_t e =
         c.act4 ? cudaLaunchKernelEx(&pc, k_xprep_act4, x, c.M, c.K, wsb + c.ws_x_off, c.x_pitch, emax, lo,
-                                    reinterpret_cast<float*>(wsb + c.ws_xmeta_off + 128))
-               : cudaLaunchKernelEx(&pc, k_xprep, x, c.M, c.K, wsb + c.ws_x_off, c.x_pitch, emax, lo);
+                                    reinterpret_cast<float*>(wsb + c.ws_xmeta_off + 64))
+               : cudaLaunchKernelEx(&pc, k_xprep, x, c.M, c.K, wsb + c.ws_x_off, c.x_pitch, emax, lo,
+                                    (c.K / KS + c.xchunks - 1) / c.xchunks);
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};

@@ -161,12 +161,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
 // Bounded wait on an mbarrier phase by one thread. Returns false if the CTA is
 // aborting or the wait ran out (then the CTA starts aborting and the status
 // word says who).
+// hint_ns > 0: the thread may sleep in hardware between probes (until the
+// phase completes or about hint_ns pass), leaving issue slots to the warps
+// that issue tensor-core work.
 __device__ __forceinline__ bool wait_bar(uint32_t b, uint32_t parity, volatile int* abort_flag,
-                                         const Params& p, uint32_t who) {
+                                         const Params& p, uint32_t who, uint32_t hint_ns = 0) {
   if (mbar_test(b, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_test(b, parity)) return true;
+    if (hint_ns ? mbar_wait_hint(b, parity, hint_ns) : mbar_test(b, parity)) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > p.timeout) {
       *abort_flag = 1;
@@ -178,9 +181,9 @@ __device__ __forceinline__ bool wait_bar(uint32_t b, uint32_t parity, volatile i
 // The same for a whole warp: lane 0 waits, the others take its answer and,
 // on success, observe the completed phase themselves.
 __device__ __forceinline__ bool warp_wait(uint32_t b, uint32_t parity, volatile int* abort_flag,
-                                          const Params& p, uint32_t who, int lane) {
+                                          const Params& p, uint32_t who, int lane, uint32_t hint_ns = 0) {
   bool ok = true;
-  if (lane == 0) ok = wait_bar(b, parity, abort_flag, p, who);
+  if (lane == 0) ok = wait_bar(b, parity, abort_flag, p, who, hint_ns);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
   if (ok && lane != 0) (void)mbar_test(b, parity);
   return ok;
@@ -325,7 +328,7 @@ k_tc4(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
           for (int j = 0; j < q.cnt; ++j, ++n_issued) {
             const int st = int(n_issued % NST);
             const uint32_t ph = uint32_t(n_issued / NST) & 1u;
-            if (!wait_bar(b_empty + 8 * st, ph ^ 1u, abort_flag, p, ST_TIMEOUT_PRODUCER)) { stop = true; break; }
+            if (!wait_bar(b_empty + 8 * st, ph ^ 1u, abort_flag, p, ST_TIMEOUT_PRODUCER, 1000)) { stop = true; break; }
             uint8_t* sb = smem + st * STAGE;
             mbar_expect_tx(b_full + 8 * st, W_BYTES + S_BYTES + XB_BYTES);
             tma_load_2d_hint(smem_u32(sb), &tm_w, (q.ks0 + j) * (KS / 2), q.tile * TROWS, b_full + 8 * st, pol);
@@ -475,7 +478,8 @@ k_tc4(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
       const Unit q = unit_of(p, u);
       const int ab = tcount & 1;
       // the eight warps agree on every outcome, so none waits alone at a barrier below
-      const bool ok = warp_wait(b_accf + 8 * ab, uint32_t(tcount >> 1) & 1u, abort_flag, p, ST_TIMEOUT_EPI, lane);
+      const bool ok =
+          warp_wait(b_accf + 8 * ab, uint32_t(tcount >> 1) & 1u, abort_flag, p, ST_TIMEOUT_EPI, lane, 20000);
       if (!named_bar_and(BAR_EPI, NUM_EPI * 32, ok)) break;
       fence_after();
       uint32_t v[16];

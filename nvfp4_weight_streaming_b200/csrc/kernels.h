@@ -82,6 +82,7 @@ struct MmaConfig {
   // X in the ring (M > 4): X planes prepared once per call in the workspace
   bool xr;
   int x_pitch, x_box, xbytes;
+  int xchunks;   // X-conversion blocks per token (grid M x xchunks)
   size_t ws_x_off, ws_xmeta_off;
   size_t smem, ws_counters_off, ws_epi_off, ws_partials_off, ws_bytes;
 };
