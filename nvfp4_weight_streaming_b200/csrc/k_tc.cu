@@ -65,9 +65,14 @@ constexpr int D_COLS = 64;               // columns per accumulator buffer (2 bu
 // serialise on it, independent ones overlap. The epilogue adds them.
 
 constexpr int TMEM_COLS = 512;
-constexpr int NUM_WARPS = 14;
+// warp 0 producer, warps 1-2 MMA issuers (a tcgen05.mma holds its issuing
+// thread for ~100+ cycles, so one thread cannot issue a stage's 16 MMAs at
+// the stream rate; each warp owns half of the accumulators), 3-10 decoders,
+// 11-14 epilogue
+constexpr int NUM_WARPS = 15;
 constexpr int NUM_THREADS = NUM_WARPS * 32;
-constexpr int WARP_DEC0 = 2, NUM_DEC = 8, WARP_EPI0 = 10, NUM_EPI = 4;
+constexpr int WARP_MMA0 = 1, NMW = 2;
+constexpr int WARP_DEC0 = 3, NUM_DEC = 8, WARP_EPI0 = 11, NUM_EPI = 4;
 constexpr int X_BUDGET = 96 * 1024;      // bytes of resident X slice
 constexpr int LO_SHIFT = 29;             // lo plane scale relative to hi
 
@@ -239,9 +244,9 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NSTAGE; ++i) { mbar_init(b_full + 8 * i, 1); mbar_init(b_empty + 8 * i, NUM_DEC); }
-    for (int i = 0; i < TSTAGE; ++i) { mbar_init(b_afull + 8 * i, NUM_DEC); mbar_init(b_aempty + 8 * i, 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(b_dfull + 8 * i, 1); mbar_init(b_dempty + 8 * i, NUM_EPI); }
-    mbar_init(b_done, 1);
+    for (int i = 0; i < TSTAGE; ++i) { mbar_init(b_afull + 8 * i, NUM_DEC); mbar_init(b_aempty + 8 * i, NMW); }
+    for (int i = 0; i < 2; ++i) { mbar_init(b_dfull + 8 * i, NMW); mbar_init(b_dempty + 8 * i, NUM_EPI); }
+    for (int i = 0; i < NMW; ++i) mbar_init(b_done + 8 * i, 1);
     misc[1] = 0; misc[2] = 0; misc[3] = 0;
     for (int m = 0; m < 16; ++m) emax[m] = INT_MIN;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -361,8 +366,10 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
     const int n_mma = (p.M <= 8) ? 16 : (need_lo ? 32 : 16);
     const int nacc = D_COLS / n_mma;
 
-    if (warp == 1) {
-      // ---------------------------------------------------------- MMA issuer
+    if (warp < WARP_DEC0) {
+      // ---------------------------------------------------------- MMA issuers
+      // warp w issues the MMAs of the accumulators a with a % NMW == w
+      const int mw = warp - WARP_MMA0;
       if (lane == 0) {
         const uint32_t idesc = (1u << 4) | (uint32_t(n_mma >> 3) << 17) | (uint32_t(ROWS >> 4) << 24);
         const uint32_t x_base = smem_u32(sX);
@@ -387,6 +394,7 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
             fence_after();
 #pragma unroll
             for (int kk = 0; kk < KC / 16; ++kk) {
+              if ((kk % nacc) % NMW != mw) continue;
               const uint32_t a_tmem = tmem + ts * A_COLS + kk * 8;
               const uint64_t bd = smem_desc(x_base + uint32_t(j * KC + kk * 16) * 16u, 128u, sbo);
               const int acc_i = kk % nacc;
@@ -400,8 +408,8 @@ k_tc(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorM
           ++sidx;
         }
         // all MMAs issued by this thread complete before tensor memory is freed
-        mma_commit(b_done);
-        drain_bar(b_done, 0u, p);
+        mma_commit(b_done + 8 * mw);
+        drain_bar(b_done + 8 * mw, 0u, p);
       }
       __syncwarp();   // reconverge warp 1 before the block barrier and dealloc
     } else if (warp < WARP_EPI0) {
