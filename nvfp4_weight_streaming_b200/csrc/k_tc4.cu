@@ -198,6 +198,26 @@ __device__ __forceinline__ void drain_bar(uint32_t b, uint32_t parity, const Par
   }
 }
 
+// Sum of the S slices' fp32 partials of row r for tokens m < M, each token's
+// sum in slice order: G slices x MT tokens of loads in flight per round (the
+// loads of a thread would otherwise wait on one another through the adds).
+template <int MT, int G>
+__device__ __forceinline__ void sum_slices(const float* base, int S, int M, int r, float* sum) {
+  for (int s0 = 0; s0 < S; s0 += G) {
+    float v[G][MT];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        v[g][m] = (s0 + g < S && m < M) ? __ldcg(base + (size_t(s0 + g) * M + m) * TROWS + r) : 0.0f;
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int m = 0; m < MT; ++m)
+        if (s0 + g < S) sum[m] += v[g][m];
+  }
+}
+
 struct Unit {
   int tile, slice, ks0, cnt;
 };
@@ -273,7 +293,10 @@ k_x4_quant(const uint16_t* __restrict__ x, int M, int K, const uint32_t* __restr
 
 // ---- the kernel -------------------------------------------------------------
 
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+// At most 96 registers: 4 warps of one SM sub-partition then leave 4096 of
+// its 16384 registers to the next call's X kernels (2 warps of <= 40), which
+// start on these SMs while this grid runs (programmatic dependent launch).
+__global__ void __maxnreg__(96)
 k_tc4(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -513,11 +536,14 @@ k_tc4(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensor
           __threadfence();
           if (row < p.N) {
             const float* base = p.partials + size_t(q.tile) * p.S * size_t(p.M) * TROWS;
-            for (int m = 0; m < p.M; ++m) {
-              float sum = 0.0f;
-              for (int s = 0; s < p.S; ++s) sum += __ldcg(base + (size_t(s) * p.M + m) * TROWS + r);
-              p.y[size_t(m) * p.N + row] = float_to_bf16_bits(__fmul_rn(scale, sum));
-            }
+            float sum[NTOK];
+#pragma unroll
+            for (int m = 0; m < NTOK; ++m) sum[m] = 0.0f;
+            if (p.M <= 4) sum_slices<4, 8>(base, p.S, p.M, r, sum);
+            else sum_slices<NTOK, 2>(base, p.S, p.M, r, sum);
+#pragma unroll
+            for (int m = 0; m < NTOK; ++m)
+              if (m < p.M) p.y[size_t(m) * p.N + row] = float_to_bf16_bits(__fmul_rn(scale, sum[m]));
           }
         }
         named_bar(BAR_EPI, NUM_EPI * 32);
