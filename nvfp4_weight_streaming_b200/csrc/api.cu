@@ -500,8 +500,12 @@ nvfp4_status nvfp4_linear_run_static(nvfp4_plan_t plan, const uint8_t* w_packed,
   size_t zeroed = plan->ws_bytes;
   if (plan->variant == int(NVFP4_VARIANT_MMA) && plan->mma.ws_partials_off < zeroed)
     zeroed = plan->mma.ws_partials_off;
-  if (plan->variant == int(NVFP4_VARIANT_TC) && plan->tc.ws_partials_off < zeroed)
+  if (plan->variant == int(NVFP4_VARIANT_TC) && !plan->act4 && plan->tc.ws_partials_off < zeroed)
     zeroed = plan->tc.ws_partials_off;
+  // W4A4 on the FP4 tensor cores: status word, X amax, gs_x and counters lie
+  // before the X blocks
+  if (plan->variant == int(NVFP4_VARIANT_TC) && plan->act4 && plan->tc4.ws_x_off < zeroed)
+    zeroed = plan->tc4.ws_x_off;
   if (plan->variant == int(NVFP4_VARIANT_ROW) && plan->row.ws_partials_off < zeroed)
     zeroed = plan->row.ws_partials_off;
   if (zeroed > 0 && cudaMemsetAsync(scratch, 0, zeroed, st) != cudaSuccess) return NVFP4_ERR_CUDA;

@@ -107,6 +107,74 @@ def test_static_scratch_recovers_after_a_timed_out_run(variant):
         nv.nvfp4_linear_destroy(plan)
 
 
+W4A4_TC = nv.NVFP4_PLAN_ACT_NVFP4 | nv.NVFP4_VARIANT_TC
+
+
+def _w4a4_ref(w, X):
+    M, K = X.shape
+    xp, xs, gsx = oracle.quantize_x(X)
+    return oracle.linear_w4a4(w.packed_h, w.scales_h, w.gs, xp, xs, gsx, M, w.N, K)
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 1024, 8192), (1, 5120, 17408), (5, 300 * 256, 512)])
+def test_static_scratch_w4a4_tensor_cores(M, N, K):
+    """W4A4 on the FP4 tensor cores: the X blocks, the X amax and the K-split
+    partials in the fixed array; bit-identical to the workspace entry."""
+    w, X = _problem(M, N, K, seed=31 + M)
+    y_ref, ad = _w4a4_ref(w, X)
+    plan = nv.nvfp4_linear_plan(M, N, K, torch.cuda.current_device(), W4A4_TC)
+    try:
+        assert nv.nvfp4_linear_variant(plan) == nv.NVFP4_VARIANT_TC
+        assert nv.nvfp4_linear_workspace_bytes(plan) <= nv.NVFP4_STATIC_SCRATCH_BYTES
+        y_ws, ok, _ = run_linear(w, X, plan=plan)
+        assert ok
+        check_tolerance(y_ws, y_ref, ad)
+        xd = dev(X)
+        status = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+        outs = []
+        for call in range(2):
+            y = Guarded(M * N)
+            nv.nvfp4_linear_run_static(plan, w.packed, w.scales, w.gsd, xd, y.view, status[call:call + 1])
+            outs.append(y)
+        torch.cuda.synchronize()
+        assert status.tolist() == [0, 0]
+        for y in outs:
+            assert y.guards_intact()
+            assert (host_u16(y.view).reshape(M, N) == y_ws).all()
+    finally:
+        nv.nvfp4_linear_destroy(plan)
+
+
+def test_static_scratch_w4a4_recovers_after_a_timed_out_run():
+    """A stalled W4A4 tensor-core plan leaves its status and possibly counters
+    in the shared array; the next static call clears them and is right."""
+    M, N, K = 1, 5120, 17408                       # K split: per-tile counters in use
+    w, X = _problem(M, N, K, seed=41)
+    y_ref, ad = _w4a4_ref(w, X)
+    dev_id = torch.cuda.current_device()
+    xd = dev(X)
+    status = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    stalled = nv.nvfp4_linear_plan(M, N, K, dev_id, W4A4_TC | nv.NVFP4_PLAN_TEST_STALL)
+    try:
+        y = Guarded(M * N)
+        nv.nvfp4_linear_run_static(stalled, w.packed, w.scales, w.gsd, xd, y.view, status[0:1])
+        torch.cuda.synchronize()
+        assert int(status[0].item()) != 0
+        assert y.guards_intact()
+    finally:
+        nv.nvfp4_linear_destroy(stalled)
+    plan = nv.nvfp4_linear_plan(M, N, K, dev_id, W4A4_TC)
+    try:
+        y = Guarded(M * N)
+        nv.nvfp4_linear_run_static(plan, w.packed, w.scales, w.gsd, xd, y.view, status[1:2])
+        torch.cuda.synchronize()
+        assert int(status[1].item()) == 0
+        assert y.guards_intact()
+        check_tolerance(host_u16(y.view).reshape(M, N), y_ref, ad)
+    finally:
+        nv.nvfp4_linear_destroy(plan)
+
+
 def test_static_scratch_rejects_plans_beyond_its_size():
     """A plan whose workspace exceeds the fixed array is refused with
     WORKSPACE and launches nothing."""
