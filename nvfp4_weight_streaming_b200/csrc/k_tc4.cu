@@ -41,6 +41,8 @@
 // 32 x 128 bits broadcast to the four quadrants writes exactly that from a
 // 512-byte shared-memory atom whose byte 16 * m0 + 4 * m1 + b is block b of
 // row 32 * m1 + m0. The token scales use the same atom (tokens < 16: m1 = 0).
+// So each MMA's scales take 4 columns, and every scale address an MMA is
+// given is a multiple of 4 columns.
 //
 // Work split: units are (256-row tile, K-slice) pairs. When the tiles fill
 // the SMs a unit is a whole tile and CTAs loop over tiles; otherwise K is cut
