@@ -30,6 +30,9 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+# calls per timed block of a sweep point (the headline uses --steps): a few
+# seconds of timed work even for the 715 MB lm_head
+SWEEP_CALLS = 2000
 METRIC = "NVFP4 linear effective HBM GB/s and % of peak at M=1/16 (27B-class shapes)"
 NOMINAL_HBM_GBS = 8000.0
 VARIANT_NAMES = ("auto", "gemv", "mma", "tc", "row")
@@ -431,9 +434,10 @@ def run_ours(args):
     value = effective_gbs(pb.bytes * world, sec)
     per_gpu = effective_gbs(pb.bytes, sec)
     sweep = []
-    if not args.no_sweep:
+    if not args.no_sweep and world == 1:
         # every workload shape and M (the down projection's 64 rotated copies
-        # included), then the fused epilogues and the FP8 comparison tier
+        # included), then the fused epilogues and the FP8 comparison tier;
+        # single-GPU runs only, SWEEP_CALLS calls per timed block
         points = [("verify", m, "nvfp4", "none") for m in (1, 2, 4, 8, 12, 16)] + \
                  [("down", m, "nvfp4", "none") for m in (1, 4, 8, 16)] + \
                  [("lm_head", m, "nvfp4", "none") for m in (1, 8, 16)] + \
@@ -452,7 +456,8 @@ def run_ours(args):
         for (name, M, fmt, epi, forced) in points:
             v = forced if forced is not None else variant if (fmt == "nvfp4" and epi == "none") else 0
             q = Problem(name, M, v, min_footprint=4.2 * l2, flags=flags, fmt=fmt, epi=epi)
-            s2, _, r2 = time_problem(q, max(args.steps, 200), args.warmup, world, repeats=args.repeats)
+            s2, _, r2 = time_problem(q, max(min(args.steps, SWEEP_CALLS), 200), args.warmup, world,
+                                     repeats=args.repeats)
             g = effective_gbs(q.bytes, s2)
             pt = {"workload": name, "M": M, "N": q.N, "K": q.K,
                   "weights": "nvfp4" if fmt == "w4a4" else fmt,
