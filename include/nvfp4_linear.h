@@ -114,9 +114,9 @@ typedef struct nvfp4_plan_s* nvfp4_plan_t;
  * codes, one byte per element, with one fp32 scale per row, for comparison
  * with NVFP4 at the same shapes (page "Qwen3.8-27B-NVFP4-RTX5090 API &
  * Inference Endpoint", section "Measured against the other NVFP4 builds of
- * this model": the next instruction tier costs 1.5-2.1x on these GEMM
- * shapes; page "InventDB Sparkle", section "How it answers quickly": 8-bit
- * weights). With this flag w_packed is uint8 [N][K] (E4M3 codes), w_scales
+ * this model": a weight format one step wider than NVFP4 is reported 1.5 to
+ * 2.1 times slower on these shapes; page "InventDB Sparkle", section "How it
+ * answers quickly": 8-bit weights). With this flag w_packed is uint8 [N][K] (E4M3 codes), w_scales
  * is float [N] and w_hat[n][k] = e4m3(code[n][k]) * w_scales[n] * gs; X, Y,
  * the tolerance and the X range are as for NVFP4. nvfp4_quantize_fp8 makes
  * such weights. */
